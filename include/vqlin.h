@@ -1,0 +1,219 @@
+/*
+ * vqlin.h — C ABI of libvqlin, a linear layer that runs directly on
+ * vector-quantised (VQ) weights with a sparse outlier correction, for
+ * NVIDIA B200 (sm_100a).
+ *
+ * What one layer computes
+ * -----------------------
+ * The weight W is n_out x n_in (row = output feature, the usual Linear
+ * layout).  It is never stored densely.  Instead:
+ *
+ *   - the columns of W are split into the "main" columns and an optional,
+ *     caller-chosen set of "outlier columns" (VPTQ: Extreme Low-bit Vector
+ *     Post-Training Quantization for Large Language Models, section
+ *     "Outlier Elimination": a separate codebook for a few percent of the
+ *     columns, decoded through a static branch);
+ *   - each row's main columns, taken in increasing column order, are cut into
+ *     sub-vectors of d consecutive elements; sub-vector s of row i is the
+ *     codebook entry C1[i1] (plus C2[i2] when a residual codebook is given:
+ *     VPTQ page, section "Residual Vector Quantization", "Decoding process");
+ *   - each row's outlier columns, in increasing column order, are cut the same
+ *     way and decoded with their own codebook Co;
+ *   - every element is multiplied by a row scale r[i] and a column scale c[j]
+ *     (SCVQ: Sparse-Compensated Vector Quantization for Large Language Models,
+ *     summary, step 1 "bi-normalized across rows and columns"; the stored
+ *     scales are multipliers at decode time);
+ *   - a sparse CSR matrix S gives exact values for chosen positions:
+ *     W[i,j] = v_ij for (i,j) in S (HAS-VQ: Hessian-Adaptive Sparse Vector
+ *     Quantization for High-Fidelity LLM Compression, abstract: the sparse
+ *     feedback makes outliers reconstruct exactly; SCVQ summary, step 4: one
+ *     sparse correction matrix).  Positions in S take precedence over the
+ *     outlier block, which takes precedence over the main body.
+ *
+ *   So, for (i,j) not in S:
+ *     W[i,j] = r[i] * c[j] * Co[io(i, p/d)][p % d]                 if j is the p-th outlier column
+ *     W[i,j] = r[i] * c[j] * (C1[i1(i,q/d)] + C2[i2(i,q/d)])[q % d] if j is the q-th main column
+ *   (no residual codebook: the C2 term is absent, not +0; no scale: factor 1).
+ *
+ * The layer then computes y[b,:] = W x[b,:] (decode, batch 1..16) or
+ * Y = X W^T (prefill), with the dequantisation fused into the product
+ * (VPTQ page, "The dequantization interface": dequantisation fused into the
+ * GEMV for decoding and the GEMM for prefill, so the fp16 weight is never
+ * written and re-read).
+ *
+ * Packed index format
+ * -------------------
+ * A field is w = bits1 + bits2 bits wide (bits2 = 0 without a residual
+ * codebook).  Row i of the code matrix starts at byte i * row_stride_bytes.
+ * Field s of a row occupies bits [s*w, s*w + w) of that row's byte string,
+ * least significant bit first, bytes in increasing address order (so byte b
+ * holds bits 8b..8b+7, bit 0 = its LSB).  Within a field, i1 is the low bits1
+ * bits and i2 the next bits2 bits.  Example: w = 12+12, i1 = 0xABC,
+ * i2 = 0x123 -> bytes BC 3A 12.  Bits after the row's last field are ignored.
+ * The outlier block uses the same scheme with bits_o-bit fields.
+ * (The VPTQ page gives only "ceil(log2 k) bits per index"; the bit order and
+ * the per-row layout are this library's choice.)
+ *
+ * Sub-vectors per row: n_sub = ceil(n_main / d), n_main = n_in - n_ocols;
+ * n_sub_o = ceil(n_ocols / d).  The last sub-vector of a row may cover fewer
+ * than d real columns; its remaining elements are ignored.
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ *  - fp16/bf16 arrays are passed as uint16_t bit patterns.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *  - Every call returns a vqlin_status; nothing is thrown across the ABI and
+ *    no kernel traps.  A failed call leaves its outputs unspecified.
+ *    vqlin_last_error() gives a thread-local, human-readable detail string.
+ *  - Kernels run asynchronously on `stream`; a launch failure is reported as
+ *    VQLIN_ERR_CUDA.  The handle is immutable after vqlin_create, so calls on
+ *    different streams may run concurrently.
+ */
+#ifndef VQLIN_H
+#define VQLIN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define VQLIN_ABI_VERSION 1
+#define VQLIN_MAX_BATCH 16
+
+typedef enum {
+  VQLIN_OK = 0,
+  VQLIN_ERR_INVALID_ARG = 1,  /* NULL pointer, bad size, bad stride or alignment   */
+  VQLIN_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. d not in {4,8})    */
+  VQLIN_ERR_INVALID_DATA = 3, /* index >= k, malformed CSR, non-finite value        */
+  VQLIN_ERR_OOM = 4,          /* device or host allocation failed                   */
+  VQLIN_ERR_CUDA = 5,         /* a CUDA call or kernel launch failed                */
+  VQLIN_ERR_WORKSPACE = 6     /* workspace NULL, too small or misaligned            */
+} vqlin_status;
+
+typedef enum { VQLIN_F32 = 0, VQLIN_F16 = 1, VQLIN_BF16 = 2 } vqlin_dtype;
+
+typedef struct vqlin_handle vqlin_handle;
+
+/*
+ * Layer description.  Pointers are borrowed for the duration of vqlin_create
+ * only; they are device pointers unless src_on_host is non-zero, in which
+ * case they are host pointers.
+ */
+typedef struct {
+  int32_t n_out, n_in;        /* W is n_out x n_in; both >= 1                         */
+  int32_t d;                  /* sub-vector length; kernels support 4 and 8            */
+  int32_t src_on_host;        /* 0: pointers below are device pointers; 1: host        */
+
+  /* main body */
+  int32_t k1, bits1;          /* entries of C1 (1 <= k1 <= 2^bits1), 1 <= bits1 <= 16  */
+  int32_t k2, bits2;          /* residual C2: k2 = bits2 = 0 for none; else k2 <= 2^bits2,
+                                 1 <= bits2 <= 16 and bits1 + bits2 <= 32              */
+  const void* codes;          /* n_out rows of packed fields (format above)           */
+  int64_t row_stride_bytes;   /* >= ceil(n_sub * (bits1+bits2) / 8)                    */
+  const uint16_t* codebook1;  /* fp16 [k1][d], row-major                              */
+  const uint16_t* codebook2;  /* fp16 [k2][d] or NULL when k2 == 0                    */
+
+  /* scales (SCVQ bi-normalisation); NULL means all ones */
+  const uint16_t* row_scale;  /* fp16 [n_out]                                          */
+  const uint16_t* col_scale;  /* fp16 [n_in]                                           */
+
+  /* outlier-column block (VPTQ "Outlier Elimination"); n_ocols = 0 for none */
+  int32_t n_ocols;            /* 0 <= n_ocols <= n_in                                  */
+  const int32_t* ocols;       /* strictly increasing column ids in [0, n_in)           */
+  int32_t ko, bits_o;         /* entries of Co (ko <= 2^bits_o), 1 <= bits_o <= 16     */
+  const uint16_t* codebook_o; /* fp16 [ko][d] (the block uses the layer's d)           */
+  const void* codes_o;        /* n_out rows of packed bits_o-bit fields                */
+  int64_t o_row_stride_bytes; /* >= ceil(n_sub_o * bits_o / 8)                         */
+
+  /* sparse correction, CSR, REPLACE semantics: W[i,j] = values[e] exactly */
+  int64_t nnz;                /* 0 <= nnz; nnz = 0 allows NULL arrays                 */
+  const int32_t* row_ptr;     /* [n_out + 1], row_ptr[0] = 0, non-decreasing, = nnz at end */
+  const int32_t* col_idx;     /* [nnz], strictly increasing within a row, in [0, n_in) */
+  const uint16_t* values;     /* fp16 [nnz], finite                                    */
+} vqlin_desc;
+
+/* Sizes and bit accounting of a created layer. */
+typedef struct {
+  int32_t n_out, n_in, d, n_sub, n_sub_o, n_ocols;
+  int64_t nnz;
+  int64_t index_bytes;        /* packed main + outlier fields, rows packed without padding */
+  int64_t codebook_bytes;     /* 2 * d * (k1 + k2 + ko)                                 */
+  int64_t scale_bytes;        /* 2 * (n_out if row scales) + 2 * (n_in if column scales) */
+  int64_t sparse_bytes;       /* CSR: nnz * (2 value + 4 column) + 4 * (n_out + 1)      */
+  /* VPTQ page, "Compression ratio calculation": original fp16 bits divided by
+     (codebook bits + index bits); equivalent bit width = 16 / ratio.  These two
+     use exactly that formula (main codebook and main indices only). */
+  double vptq_compression_ratio;
+  double vptq_bits_per_weight;
+  /* everything the layer stores (indices, all codebooks, scales, CSR), in bits per weight */
+  double total_bits_per_weight;
+} vqlin_info;
+
+/*
+ * Validate `desc`, copy and repack everything into device memory owned by the
+ * returned handle, and synchronise `stream` before returning.
+ * Checks: shapes and bit widths; CSR structure, column range, ordering and
+ * finiteness; codebook and scale finiteness; ocols ordering; every decoded
+ * index < its k.  Errors: INVALID_ARG, UNSUPPORTED, INVALID_DATA, OOM, CUDA.
+ * On error *out is set to NULL.
+ */
+vqlin_status vqlin_create(const vqlin_desc* desc, void* stream, vqlin_handle** out);
+
+/* Free the handle's device memory.  NULL is accepted.  The caller must make sure
+   no call using the handle is still running. */
+vqlin_status vqlin_destroy(vqlin_handle* h);
+
+vqlin_status vqlin_get_info(const vqlin_handle* h, vqlin_info* info);
+
+/*
+ * Dense fp16 weight: W[i*ldw + j] for 0 <= i < n_out, 0 <= j < n_in, written
+ * on `stream` (device pointer, ldw >= n_in).  Each element is the IEEE fp16
+ * value nearest (ties to even; overflow to +-inf) to the exact real value of
+ * the formula above; at CSR positions it is v_ij bit for bit.  Zero results
+ * carry the sign IEEE arithmetic gives r*c*(C1 + C2) (C1 alone without C2).
+ * (VPTQ page, "The dequantization interface": W = C[indices] and
+ * C[indices1] + Cres[indices2].)
+ */
+vqlin_status vqlin_dequant(const vqlin_handle* h, uint16_t* W, int64_t ldw, void* stream);
+
+/*
+ * Decode (VPTQ page: "QGemv", dequantisation fused into the GEMV):
+ *   y[b*n_out + i] = sum_j W[i,j] * x[b*n_in + j],  0 <= b < batch <= 16.
+ * x: device [batch][n_in] of xt (F16, BF16 or F32); y: device [batch][n_out]
+ * of yt.  Products and sums are fp32 (W's unrounded value r*c*C enters through
+ * fp32 arithmetic, not through an fp16 weight).  x and y must be 16-byte
+ * aligned and must not overlap.  Summation order is unspecified.
+ */
+vqlin_status vqlin_gemv(const vqlin_handle* h, const void* x, vqlin_dtype xt, int32_t batch,
+                        void* y, vqlin_dtype yt, void* stream);
+
+/*
+ * Prefill: Y[m*n_out + i] = sum_j W[i,j] * X[m*n_in + j] for 0 <= m < M.
+ * X: device [M][n_in] of xt (F16 or BF16; BF16 is converted to fp16, exact for
+ * 2^-14 <= |x| <= 65504), Y: device [M][n_out] of yt.  The weight enters the
+ * tensor-core product as its fp16 dequantised value; accumulation is fp32.
+ * workspace: device memory of at least vqlin_gemm_workspace_size(h, M) bytes,
+ * 256-byte aligned, owned by the caller, not used concurrently by another call.
+ * Errors additionally: WORKSPACE, UNSUPPORTED (M < 1 or n_in % 8 != 0).
+ */
+vqlin_status vqlin_gemm(const vqlin_handle* h, const void* X, vqlin_dtype xt, int64_t M,
+                        void* Y, vqlin_dtype yt, void* workspace, size_t ws_bytes, void* stream);
+size_t vqlin_gemm_workspace_size(const vqlin_handle* h, int64_t M);
+
+/*
+ * Test hook: decoded fields.  which = 0: main body, out[i*n_sub + s] =
+ * i1 | (i2 << bits1); which = 1: outlier block, out[i*n_sub_o + s].
+ * `out` is a device uint32 array.
+ */
+vqlin_status vqlin_unpack_indices(const vqlin_handle* h, int32_t which, uint32_t* out, void* stream);
+
+const char* vqlin_status_string(vqlin_status s);
+const char* vqlin_last_error(void);
+int32_t vqlin_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VQLIN_H */

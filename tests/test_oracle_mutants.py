@@ -1,0 +1,47 @@
+"""The oracle's pins catch plausible mistakes (CPU only).
+
+Each case copies oracle.c, plants one mistake (a dropped or sign-flipped term,
+a wrong index, a transposed operand, a wrong rounding rule, a wrong bit order),
+builds the copy, and runs the pin suite against it: the suite must fail.
+"""
+import os
+import shutil
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "oracle.c")
+
+MUTANTS = {
+    "residual_sign": ("v = v + oracle_f16_to_f64(*e2);", "v = v - oracle_f16_to_f64(*e2);"),
+    "residual_dropped_exact": ("  if (h2) {\n    int s2, e2;", "  if (0) {\n    int s2, e2;"),
+    "ties_away": ("if (rem > half || (rem == half && (N & 1))) N += 1;", "if (rem >= half) N += 1;"),
+    "msb_first": ("uint32_t b = (row[bit >> 3] >> (bit & 7)) & 1u;", "uint32_t b = (row[bit >> 3] >> (7 - (bit & 7))) & 1u;"),
+    "element_reversed": ("*e1 = L->cb1 + (int64_t)i1 * d + (q % d);", "*e1 = L->cb1 + (int64_t)i1 * d + (d - 1 - q % d);"),
+    "replace_dropped": ("W[(int64_t)i * ldw + L->col_idx[e]] = L->values[e];   /* REPLACE: exact outliers */", ";"),
+    "operand_reversed": ("for (int32_t j = 0; j < L->n_in; ++j) acc += w[j] * x[j];",
+                         "for (int32_t j = 0; j < L->n_in; ++j) acc += w[j] * x[L->n_in - 1 - j];"),
+    "subnormal_exponent": ("if (e == 0) { *mant = f; *exp2 = -24; }", "if (e == 0) { *mant = f; *exp2 = -25; }"),
+    "outlier_codebook": ("*e1 = L->cbo + (int64_t)io * d + (p % d);",
+                         "*e1 = L->cb1 + (int64_t)(io % L->k1) * d + (p % d);"),
+    "col_scale_dropped": ("if (L->cs) v = v * oracle_f16_to_f64(L->cs[j]);", ";"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_fail_on_planted_mistake(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, "mutation site not found: " + name
+    mutant_c = tmp_path / "oracle_mutant.c"
+    mutant_c.write_text(src.replace(old, new))
+    lib = tmp_path / "liboracle_mutant.so"
+    subprocess.check_call(["gcc", "-O2", "-std=gnu99", "-ffp-contract=off", "-fPIC", "-shared",
+                           str(mutant_c), "-o", str(lib), "-lm"])
+    env = dict(os.environ, VQ_ORACLE_LIB=str(lib))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, "pins did not notice mutant %s:\n%s" % (name, r.stdout[-2000:])
