@@ -1,0 +1,426 @@
+#!/usr/bin/env python3
+"""Benchmark of the VQ + sparse linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl vqlin|reference]
+                    [--config qproj|tiny|downproj|smollm|prefill] [--batch B]
+
+Default workload: the LLaMA-2-7B q_proj-shaped layer (4096x4096, d=8,
+K=65536 fp16 codebook = 2 bits/weight, row and column scales, 1% CSR outliers),
+batch-1 decode GEMV, fp16 x and y.  One step = one pass of the hot path
+(one vqlin_gemv call; for `smollm` the seven linears of a decoder layer back to
+back; for `prefill` one vqlin_gemm call).
+
+Timing: W untimed eager steps, then the K steps are captured in one CUDA graph
+(replayed once untimed to upload it) and replayed once between CUDA events on
+the launching stream, with a barrier and a device synchronisation on both
+sides; the maximum over ranks is reported.  Weights rotate through enough
+independent copies to exceed 3x the L2 size, so every step streams its weights
+from HBM.  SM clocks and throttle reasons are sampled through NVML during the
+timed region.  `e2e` repeats the K steps eagerly through the same C-ABI calls
+with the step's input copied from pinned host memory and its output read back
+to pinned host memory (stream synchronised) every step.
+
+One JSON line is printed by rank 0.  Under torchrun (N > 1) every rank runs an
+independent replica (the layer shards by rows with no exchange; here each rank
+runs the whole layer): scaling is weak and value sums the ranks' bytes over the
+slowest rank's time.
+
+--impl reference times the CPU oracle on the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_compensated_vq_b200 import synth  # noqa: E402
+
+METRIC = "VQ+sparse GEMV us/call & HBM GB/s (% of B200 peak), 4096x4096 2-bit, batch 1"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+# --------------------------------------------------------------------------- workloads
+class Workload:
+    def __init__(self, name, layers, xs, calls, kind, desc):
+        self.name, self.layers, self.xs, self.calls, self.kind, self.desc = name, layers, xs, calls, kind, desc
+
+    def weight_bytes(self):
+        return sum(L.abi_bytes()["total"] for L in self.layers)
+
+    def io_bytes(self):
+        b = 0
+        for (li, B) in self.calls:
+            L = self.layers[li]
+            xb = self.xs[li]
+            b += xb[:B].nbytes + B * L.n_out * 2        # x in its dtype, y fp16/bf16
+        return b
+
+    def bytes_per_step(self):
+        return self.weight_bytes() + self.io_bytes()
+
+    def flops_per_step(self):
+        return sum(2.0 * self.layers[li].n_out * self.layers[li].n_in * B for li, B in self.calls)
+
+
+def make_workload(name: str, batch: int) -> Workload:
+    if name == "qproj":
+        L, xb = synth.qproj(batch)
+        return Workload("llama2_7b_qproj_4096x4096_d8_k65536_2bit_b%d" % batch, [L], [xb], [(0, batch)], "gemv",
+                        "4096x4096, d=8, K=65536 fp16 codebook (16-bit codes, 2 bits/weight), fp16 row+col scales, "
+                        "1%% CSR outliers, fp16 x/y, batch %d" % batch)
+    if name == "tiny":
+        L, xb = synth.tiny()
+        return Workload("tiny_256x256_d4_k256_b1", [L], [xb], [(0, 1)], "gemv", "256x256, d=4, K=256, 1% CSR")
+    if name == "downproj":
+        L, xb = synth.downproj(batch)
+        return Workload("llama2_7b_downproj_4096x11008_rvq12x12_b%d" % batch, [L], [xb], [(0, batch)], "gemv",
+                        "4096x11008, d=8, residual VQ 12+12 bits, 110 outlier columns (K=256), 0.5%% CSR, batch %d" % batch)
+    if name == "smollm":
+        Ls, xs = synth.smollm(batch)
+        return Workload("smollm2_1.7b_layer_7linears_d8_k256_b%d" % batch, Ls, xs, [(i, batch) for i in range(7)],
+                        "gemv", "7 linears of a SmolLM2-1.7B layer, d=8, K=256, 2%% Hessian-style outliers, bf16 x, batch %d" % batch)
+    if name == "prefill":
+        L, Xb = synth.prefill(2048)
+        return Workload("prefill_2048x4096x4096_d8_k65536", [L], [Xb], [(0, 2048)], "gemm",
+                        "X 2048x4096 bf16 times the q_proj-shaped VQ weight, bf16 Y")
+    raise SystemExit("unknown config " + name)
+
+
+# --------------------------------------------------------------------------- helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sparse_compensated_vq_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload_name):
+    """DRAM bytes per launch from a committed ncu capture, if the kernels have not changed since."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d.get(workload_name)
+        if e and e.get("source_hash") == kernel_source_hash():
+            return e.get("dram_bytes_per_launch")
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index):
+        self.samples, self.reasons, self.err = [], 0, None
+        self.stop_flag = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # NVML missing: report, do not fail the bench
+            self.nv, self.err, self.max_mhz = None, str(e), None
+
+    def _sample(self):
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception as e:
+            self.err = str(e)
+
+    def _run(self):
+        while not self.stop_flag.is_set():
+            self._sample()
+            time.sleep(0.001)
+
+    def __enter__(self):
+        if self.nv:
+            self._sample()
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.nv:
+            self.stop_flag.set()
+            self.t.join()
+            self._sample()
+
+    def report(self):
+        if not self.nv:
+            return {"error": self.err}
+        names = [n for b, n in self.REASONS.items() if self.reasons & b]
+        return {"sm_mhz": float(np.median(self.samples)) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "samples": len(self.samples), "reasons": names}
+
+
+# --------------------------------------------------------------------------- our arm
+def run_vqlin(args, rank, world, dist):
+    import torch
+    from sparse_compensated_vq_b200 import vqlin
+
+    dev = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(dev)
+    wl = make_workload(args.config, args.batch)
+    wbytes = wl.weight_bytes()
+    n_copies = int(min(64, max(1, math.ceil(3 * L2_BYTES / wbytes))))
+    copies = [[vqlin.VQLinear(L) for L in wl.layers] for _ in range(n_copies)]
+    xdt = "bf16" if wl.name.startswith(("smollm", "prefill")) else "f16"
+    tdt = torch.bfloat16 if xdt == "bf16" else torch.float16
+
+    def dev_x(xb, B):
+        a = np.ascontiguousarray(xb[:B])
+        t = torch.from_numpy(a.view(np.int16)).cuda()
+        return t.view(tdt)
+
+    xs = [dev_x(wl.xs[li], B) for li, B in wl.calls]
+    ys = [torch.empty((B, wl.layers[li].n_out), dtype=tdt, device="cuda") for li, B in wl.calls]
+    ws = None
+    if wl.kind == "gemm":
+        ws = torch.empty(copies[0][0].workspace_size(wl.calls[0][1]), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.Stream()
+
+    def step(i, s_handle):
+        c = copies[i % n_copies]
+        for k, (li, B) in enumerate(wl.calls):
+            h = c[li].handle
+            if wl.kind == "gemv":
+                st = vqlin.vqlin_gemv(h, xs[k].data_ptr(), vqlin.dtype_code(tdt), B, ys[k].data_ptr(),
+                                      vqlin.dtype_code(tdt), s_handle)
+            else:
+                st = vqlin.vqlin_gemm(h, xs[k].data_ptr(), vqlin.dtype_code(tdt), B, ys[k].data_ptr(),
+                                      vqlin.dtype_code(tdt), ws.data_ptr(), ws.numel(), s_handle)
+            if st != 0:
+                raise vqlin.VQLinError(st, "bench step")
+
+    # our kernels per step: one per gemv call; gemm = dequant body + sparse replace + bf16->fp16 + GEMM
+    launches_per_step = len(wl.calls) if wl.kind == "gemv" else 4
+    s_ptr = stream.cuda_stream
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i, s_ptr)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        cap = torch.cuda.current_stream().cuda_stream
+        for i in range(args.steps):
+            step(i, cap)
+    g.replay()                      # upload (untimed)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    ms_max = ms
+    if dist:
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    del g
+
+    # ---- end to end: host buffers, copies inside the timed region, result read each step
+    x_host = [torch.from_numpy(np.ascontiguousarray(wl.xs[li][:B]).view(np.int16)).pin_memory() for li, B in wl.calls]
+    y_host = [torch.empty((B, wl.layers[li].n_out), dtype=torch.int16).pin_memory() for li, B in wl.calls]
+    n_e2e = args.steps
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        f0.record(stream)
+        for i in range(n_e2e):
+            for k in range(len(wl.calls)):
+                xs[k].view(torch.int16).copy_(x_host[k], non_blocking=True)
+            step(i, s_ptr)
+            for k in range(len(wl.calls)):
+                y_host[k].copy_(ys[k].view(torch.int16), non_blocking=True)
+            stream.synchronize()
+        f1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1)
+    if dist:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = sum(x.numel() * 2 for x in x_host)
+    d2h = sum(y.numel() * 2 for y in y_host)
+
+    hbm_peak, bf16_peak, bf16_sust, peak_src = load_peaks()
+    bytes_step = wl.bytes_per_step()
+    flops_step = wl.flops_per_step()
+    sec_step = ms_max / 1e3 / args.steps
+    value = world * bytes_step / sec_step / 1e9                   # GB/s, whole job
+    per_launch_s = ms / 1e3 / args.steps
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 6), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "us_per_call": round(sec_step * 1e6 / len(wl.calls), 3),
+        "config": {"workload": wl.name, "describe": wl.desc, "bytes_per_step": bytes_step,
+                   "flops_per_step": flops_step, "weight_copies": n_copies,
+                   "l2": "weights rotate through %d independent copies (%.0f MB > 3x L2)" % (n_copies, n_copies * wbytes / 1e6),
+                   "parallelism": "replicas x%d" % world},
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    if wl.kind == "gemv":
+        achieved = bytes_step / per_launch_s / 1e9
+        line["roofline"] = {"bound": "hbm", "achieved": round(achieved, 2), "peak": hbm_peak, "unit": "GB/s",
+                            "frac": round(achieved / hbm_peak, 4), "peak_source": peak_src,
+                            "traffic": recorded_traffic(wl.name),
+                            "kernel": "vqlin gemv (fused dequant + sparse + GEMV), per step of %d launch(es)" % len(wl.calls)}
+    else:
+        achieved = flops_step / per_launch_s / 1e12
+        line["roofline"] = {"bound": "tensor", "achieved": round(achieved, 2), "peak": bf16_peak, "unit": "TFLOP/s",
+                            "frac": round(achieved / bf16_peak, 4), "peak_source": peak_src + " bf16 (fp16 same rate)",
+                            "traffic": recorded_traffic(wl.name), "kernel": "vqlin gemm step (dequant + convert + GEMM)"}
+    line["e2e"] = {"value": round(world * bytes_step * n_e2e / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
+                   "us_per_step": round(e2e_ms * 1e3 / n_e2e, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    line["clocks"] = sampler.report()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_seconds)
+    for c in copies:
+        for m in c:
+            m.close()
+    return line
+
+
+# --------------------------------------------------------------------------- oracle on host cores
+def oracle_step_fn(wl: Workload, rows_per_layer):
+    import oracle
+    xs = [synth.bits_to_f64(wl.xs[li][:B], "bf16" if wl.name.startswith(("smollm", "prefill")) else "f16")
+          for li, B in wl.calls]
+    if wl.kind == "gemm":
+        xs = [x[:16] for x in xs]          # 16 of the 2048 tokens
+
+    def fn():
+        for k, (li, B) in enumerate(wl.calls):
+            oracle.gemv_f64(wl.layers[li], xs[k], rows=np.arange(rows_per_layer[li], dtype=np.int32))
+    return fn
+
+
+def sample_fraction(wl, rows_per_layer):
+    f = sum(rows_per_layer[li] / wl.layers[li].n_out for li, _ in wl.calls) / len(wl.calls)
+    if wl.kind == "gemm":
+        f *= 16 / 2048
+    return f
+
+
+def cpu_baseline(wl: Workload, budget_s=10.0):
+    rows = [L.n_out for L in wl.layers]
+    fn = oracle_step_fn(wl, rows)
+    t0 = time.perf_counter()
+    fn()
+    one = time.perf_counter() - t0
+    reps = max(1, int(budget_s / max(one, 1e-6)))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        fn()
+    per = (time.perf_counter() - t0) / reps
+    frac = sample_fraction(wl, rows)
+    value = frac * wl.bytes_per_step() / per / 1e9
+    return {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": "%d full passes of the oracle (%s) on one host core, %.2f s each; GEMM: 16 of 2048 tokens" % (
+                reps, "dequantise to double + dense matvec", per)}
+
+
+def run_reference(args, rank, world):
+    wl = make_workload(args.config, args.batch)
+    rows = [max(1, L.n_out // 64) for L in wl.layers]          # 1/64 of every layer per step
+    fn = oracle_step_fn(wl, rows)
+    for _ in range(args.warmup):
+        fn()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        fn()
+    el = time.perf_counter() - t0
+    frac = sample_fraction(wl, rows)
+    sec_step = el / args.steps
+    value = frac * wl.bytes_per_step() / sec_step / 1e9
+    sample = "each step: oracle on the first 1/64 of the rows of every layer (%s), one host core" % wl.name
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec_step * 1e3, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "describe": wl.desc, "parallelism": "rank 0 only"},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# --------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="vqlin", choices=["vqlin", "reference"])
+    ap.add_argument("--config", default="qproj", choices=["qproj", "tiny", "downproj", "smollm", "prefill"])
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return
+    dist = None
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as td
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        td.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = td
+    line = run_vqlin(args, rank, world, dist)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,415 @@
+// Host side of the libvqlin C ABI: validation, repacking, device upload,
+// bit accounting, errors and dispatch.  The arithmetic of every call runs in
+// the kernels of k_*.cu; create-time preparation runs here.
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "vqlin_internal.cuh"
+
+namespace vqlin {
+
+static thread_local std::string g_err;
+
+void set_error(const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+}
+
+vqlin_status cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return VQLIN_OK;
+  set_error("%s: %s", what, cudaGetErrorString(e));
+  return e == cudaErrorMemoryAllocation ? VQLIN_ERR_OOM : VQLIN_ERR_CUDA;
+}
+
+namespace {
+
+// fp16 bits -> double (exact); false for inf/NaN.
+bool f16_finite(uint16_t h) { return ((h >> 10) & 0x1F) != 31; }
+double f16_val(uint16_t h) { return (double)__half2float(__ushort_as_half(h)); }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+
+uint32_t host_field(const uint8_t* row, int64_t s, int w) {
+  int64_t bit = s * (int64_t)w;
+  uint64_t v = 0;
+  int nbytes = (int)(((bit & 7) + w + 7) >> 3);
+  for (int t = 0; t < nbytes; ++t) v |= (uint64_t)row[(bit >> 3) + t] << (8 * t);
+  v >>= (bit & 7);
+  return w >= 32 ? (uint32_t)v : (uint32_t)(v & ((1ull << w) - 1ull));
+}
+
+// Copy `bytes` from a caller buffer (device or host) into a host vector.
+vqlin_status fetch(const void* src, size_t bytes, bool on_host, std::vector<uint8_t>& dst, const char* what) {
+  dst.resize(bytes);
+  if (bytes == 0) return VQLIN_OK;
+  if (!src) {
+    set_error("%s is NULL", what);
+    return VQLIN_ERR_INVALID_ARG;
+  }
+  if (on_host) {
+    memcpy(dst.data(), src, bytes);
+    return VQLIN_OK;
+  }
+  return cuda_status(cudaMemcpy(dst.data(), src, bytes, cudaMemcpyDeviceToHost), what);
+}
+
+template <class T>
+const T* as(const std::vector<uint8_t>& v) { return reinterpret_cast<const T*>(v.data()); }
+
+struct Uploader {
+  vqlin_handle* h;
+  vqlin_status st = VQLIN_OK;
+  template <class T>
+  T* put(const void* src, size_t bytes, size_t pad = 16) {
+    if (st != VQLIN_OK || bytes == 0) return nullptr;
+    void* p = nullptr;
+    cudaError_t e = cudaMalloc(&p, bytes + pad);
+    if (e != cudaSuccess) { st = cuda_status(e, "cudaMalloc"); return nullptr; }
+    h->allocs[h->n_allocs++] = p;
+    e = cudaMemset(p, 0, bytes + pad);
+    if (e == cudaSuccess && src) e = cudaMemcpy(p, src, bytes, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) { st = cuda_status(e, "upload"); return nullptr; }
+    return reinterpret_cast<T*>(p);
+  }
+};
+
+}  // namespace
+}  // namespace vqlin
+
+using namespace vqlin;
+
+extern "C" {
+
+const char* vqlin_status_string(vqlin_status s) {
+  switch (s) {
+    case VQLIN_OK: return "ok";
+    case VQLIN_ERR_INVALID_ARG: return "invalid argument";
+    case VQLIN_ERR_UNSUPPORTED: return "unsupported";
+    case VQLIN_ERR_INVALID_DATA: return "invalid data";
+    case VQLIN_ERR_OOM: return "out of memory";
+    case VQLIN_ERR_CUDA: return "CUDA error";
+    case VQLIN_ERR_WORKSPACE: return "bad workspace";
+  }
+  return "unknown status";
+}
+
+const char* vqlin_last_error(void) { return g_err.c_str(); }
+int32_t vqlin_abi_version(void) { return VQLIN_ABI_VERSION; }
+
+vqlin_status vqlin_destroy(vqlin_handle* h) {
+  if (!h) return VQLIN_OK;
+  int dev = -1;
+  cudaGetDevice(&dev);
+  cudaSetDevice(h->device);
+  for (int i = 0; i < h->n_allocs; ++i) cudaFree(h->allocs[i]);
+  if (dev >= 0) cudaSetDevice(dev);
+  delete h;
+  return VQLIN_OK;
+}
+
+vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out) {
+  if (out) *out = nullptr;
+  if (!D || !out) { set_error("desc and out must not be NULL"); return VQLIN_ERR_INVALID_ARG; }
+  const bool host = D->src_on_host != 0;
+  // ---- shape checks
+  if (D->n_out < 1 || D->n_in < 1) { set_error("n_out and n_in must be >= 1"); return VQLIN_ERR_INVALID_ARG; }
+  if (D->d < 1 || D->d > 64) { set_error("d = %d out of range", D->d); return VQLIN_ERR_INVALID_ARG; }
+  if (D->d != 4 && D->d != 8) { set_error("d = %d: kernels support d in {4, 8}", D->d); return VQLIN_ERR_UNSUPPORTED; }
+  if (D->bits1 < 1 || D->bits1 > 16 || D->k1 < 1 || (int64_t)D->k1 > (1ll << D->bits1)) {
+    set_error("need 1 <= bits1 <= 16 and 1 <= k1 <= 2^bits1 (k1 = %d, bits1 = %d)", D->k1, D->bits1);
+    return VQLIN_ERR_INVALID_ARG;
+  }
+  if (D->k2 < 0 || D->bits2 < 0 || (D->k2 == 0) != (D->bits2 == 0) ||
+      (D->k2 > 0 && (D->bits2 > 16 || (int64_t)D->k2 > (1ll << D->bits2)))) {
+    set_error("residual codebook: need k2 = bits2 = 0, or 1 <= bits2 <= 16 and 1 <= k2 <= 2^bits2");
+    return VQLIN_ERR_INVALID_ARG;
+  }
+  if (D->n_ocols < 0 || D->n_ocols > D->n_in) { set_error("n_ocols out of range"); return VQLIN_ERR_INVALID_ARG; }
+  if (D->n_ocols > 0 && (D->bits_o < 1 || D->bits_o > 16 || D->ko < 1 || (int64_t)D->ko > (1ll << D->bits_o))) {
+    set_error("outlier block: need 1 <= bits_o <= 16 and 1 <= ko <= 2^bits_o");
+    return VQLIN_ERR_INVALID_ARG;
+  }
+  if (D->nnz < 0 || D->nnz > (int64_t)D->n_out * D->n_in || D->nnz > 0x7FFFFFFFll) {
+    set_error("nnz out of range");
+    return VQLIN_ERR_INVALID_ARG;
+  }
+  if (D->n_in == D->n_ocols && D->n_ocols > 0) { /* all columns in the outlier block: fine */ }
+  const int d = D->d, w = D->bits1 + D->bits2;
+  const int32_t n_main = D->n_in - D->n_ocols;
+  const int32_t n_sub = (int32_t)ceil_div(n_main, d);
+  const int32_t n_sub_o = (int32_t)ceil_div(D->n_ocols, d);
+  const int64_t row_bytes = ceil_div((int64_t)n_sub * w, 8);
+  const int64_t row_bytes_o = ceil_div((int64_t)n_sub_o * D->bits_o, 8);
+  if (n_sub > 0 && D->row_stride_bytes < row_bytes) {
+    set_error("row_stride_bytes = %lld < %lld", (long long)D->row_stride_bytes, (long long)row_bytes);
+    return VQLIN_ERR_INVALID_ARG;
+  }
+  if (n_sub_o > 0 && D->o_row_stride_bytes < row_bytes_o) {
+    set_error("o_row_stride_bytes too small");
+    return VQLIN_ERR_INVALID_ARG;
+  }
+
+  int prev_dev = 0;
+  cudaGetDevice(&prev_dev);
+  // ---- bring everything to the host
+  std::vector<uint8_t> codes, cb1, cb2, cbo, codes_o, rs, cs, ocols, rp, ci, vals;
+  vqlin_status st = VQLIN_OK;
+  if (n_sub > 0) st = fetch(D->codes, (size_t)D->row_stride_bytes * D->n_out, host, codes, "codes");
+  if (!st) st = fetch(D->codebook1, (size_t)D->k1 * d * 2, host, cb1, "codebook1");
+  if (!st && D->k2) st = fetch(D->codebook2, (size_t)D->k2 * d * 2, host, cb2, "codebook2");
+  if (!st && D->row_scale) st = fetch(D->row_scale, (size_t)D->n_out * 2, host, rs, "row_scale");
+  if (!st && D->col_scale) st = fetch(D->col_scale, (size_t)D->n_in * 2, host, cs, "col_scale");
+  if (!st && D->n_ocols) {
+    st = fetch(D->ocols, (size_t)D->n_ocols * 4, host, ocols, "ocols");
+    if (!st) st = fetch(D->codebook_o, (size_t)D->ko * d * 2, host, cbo, "codebook_o");
+    if (!st) st = fetch(D->codes_o, (size_t)D->o_row_stride_bytes * D->n_out, host, codes_o, "codes_o");
+  }
+  if (!st && D->nnz) {
+    st = fetch(D->row_ptr, (size_t)(D->n_out + 1) * 4, host, rp, "row_ptr");
+    if (!st) st = fetch(D->col_idx, (size_t)D->nnz * 4, host, ci, "col_idx");
+    if (!st) st = fetch(D->values, (size_t)D->nnz * 2, host, vals, "values");
+  }
+  if (st) return st;
+
+  // ---- validate values
+  auto finite_all = [](const std::vector<uint8_t>& v) {
+    const uint16_t* p = as<uint16_t>(v);
+    for (size_t i = 0; i < v.size() / 2; ++i) if (!f16_finite(p[i])) return false;
+    return true;
+  };
+  if (!finite_all(cb1) || !finite_all(cb2) || !finite_all(cbo) || !finite_all(rs) || !finite_all(cs)) {
+    set_error("a codebook or scale entry is inf or NaN");
+    return VQLIN_ERR_INVALID_DATA;
+  }
+  // column classification
+  std::vector<int32_t> colmap;   // main ids then outlier ids
+  std::vector<int32_t> rank(D->n_in), is_out(D->n_in, 0);
+  if (D->n_ocols) {
+    const int32_t* oc = as<int32_t>(ocols);
+    for (int32_t t = 0; t < D->n_ocols; ++t) {
+      if (oc[t] < 0 || oc[t] >= D->n_in || (t > 0 && oc[t - 1] >= oc[t])) {
+        set_error("ocols must be strictly increasing and in [0, n_in)");
+        return VQLIN_ERR_INVALID_DATA;
+      }
+      is_out[oc[t]] = 1;
+    }
+    colmap.reserve(D->n_in);
+    for (int32_t j = 0; j < D->n_in; ++j) if (!is_out[j]) colmap.push_back(j);
+    for (int32_t t = 0; t < D->n_ocols; ++t) colmap.push_back(oc[t]);
+  }
+  {
+    int32_t p = 0, q = 0;
+    for (int32_t j = 0; j < D->n_in; ++j) rank[j] = is_out[j] ? p++ : q++;
+  }
+  // indices in range (and repack rows to a 16-byte stride)
+  const int64_t stride = round_up(std::max<int64_t>(row_bytes, 1), 16);
+  const int64_t stride_o = round_up(std::max<int64_t>(row_bytes_o, 1), 16);
+  std::vector<uint8_t> codes_r((size_t)stride * D->n_out, 0), codes_o_r;
+  const uint32_t m1 = (1u << D->bits1) - 1u;
+  for (int32_t i = 0; i < D->n_out && n_sub > 0; ++i) {
+    const uint8_t* row = codes.data() + (size_t)i * D->row_stride_bytes;
+    memcpy(codes_r.data() + (size_t)i * stride, row, (size_t)row_bytes);
+    // clear the bits past the last field so the repacked rows are canonical
+    int64_t used_bits = (int64_t)n_sub * w;
+    if (used_bits & 7) codes_r[(size_t)i * stride + (used_bits >> 3)] &= (uint8_t)((1u << (used_bits & 7)) - 1u);
+    for (int32_t s = 0; s < n_sub; ++s) {
+      uint32_t f = host_field(row, s, w);
+      uint32_t i1 = f & m1, i2 = D->bits2 ? (f >> D->bits1) : 0;
+      if (i1 >= (uint32_t)D->k1 || (D->k2 && i2 >= (uint32_t)D->k2)) {
+        set_error("row %d sub-vector %d: index (%u, %u) out of range", i, s, i1, i2);
+        return VQLIN_ERR_INVALID_DATA;
+      }
+    }
+  }
+  if (D->n_ocols) {
+    codes_o_r.assign((size_t)stride_o * D->n_out, 0);
+    for (int32_t i = 0; i < D->n_out; ++i) {
+      const uint8_t* row = codes_o.data() + (size_t)i * D->o_row_stride_bytes;
+      memcpy(codes_o_r.data() + (size_t)i * stride_o, row, (size_t)row_bytes_o);
+      int64_t used_bits = (int64_t)n_sub_o * D->bits_o;
+      if (used_bits & 7) codes_o_r[(size_t)i * stride_o + (used_bits >> 3)] &= (uint8_t)((1u << (used_bits & 7)) - 1u);
+      for (int32_t s = 0; s < n_sub_o; ++s)
+        if (host_field(row, s, D->bits_o) >= (uint32_t)D->ko) {
+          set_error("row %d outlier sub-vector %d: index out of range", i, s);
+          return VQLIN_ERR_INVALID_DATA;
+        }
+    }
+  }
+  // CSR structure and the fused correction delta = v - body (double, stored fp32)
+  std::vector<float> delta((size_t)D->nnz);
+  std::vector<uint16_t> col16;
+  if (D->nnz) {
+    const int32_t* r = as<int32_t>(rp);
+    const int32_t* c = as<int32_t>(ci);
+    const uint16_t* v = as<uint16_t>(vals);
+    if (r[0] != 0 || r[D->n_out] != D->nnz) { set_error("row_ptr must start at 0 and end at nnz"); return VQLIN_ERR_INVALID_DATA; }
+    const uint16_t* C1 = as<uint16_t>(cb1);
+    const uint16_t* C2 = D->k2 ? as<uint16_t>(cb2) : nullptr;
+    const uint16_t* CO = D->n_ocols ? as<uint16_t>(cbo) : nullptr;
+    for (int32_t i = 0; i < D->n_out; ++i) {
+      if (r[i + 1] < r[i]) { set_error("row_ptr decreases at row %d", i); return VQLIN_ERR_INVALID_DATA; }
+      double ri = D->row_scale ? f16_val(as<uint16_t>(rs)[i]) : 1.0;
+      for (int32_t e = r[i]; e < r[i + 1]; ++e) {
+        int32_t j = c[e];
+        if (j < 0 || j >= D->n_in || (e > r[i] && c[e - 1] >= j)) {
+          set_error("row %d: CSR columns must be strictly increasing and in [0, n_in)", i);
+          return VQLIN_ERR_INVALID_DATA;
+        }
+        if (!f16_finite(v[e])) { set_error("CSR value %d is inf or NaN", e); return VQLIN_ERR_INVALID_DATA; }
+        double body;
+        if (is_out[j]) {
+          int32_t p = rank[j];
+          uint32_t io = host_field(codes_o.data() + (size_t)i * D->o_row_stride_bytes, p / d, D->bits_o);
+          body = f16_val(CO[(size_t)io * d + p % d]);
+        } else {
+          int32_t q = rank[j];
+          uint32_t f = host_field(codes.data() + (size_t)i * D->row_stride_bytes, q / d, w);
+          body = f16_val(C1[(size_t)(f & m1) * d + q % d]);
+          if (C2) body += f16_val(C2[(size_t)(f >> D->bits1) * d + q % d]);
+        }
+        body *= ri;
+        if (D->col_scale) body *= f16_val(as<uint16_t>(cs)[j]);
+        delta[e] = (float)(f16_val(v[e]) - body);
+      }
+    }
+    if (D->n_in <= 65536) {
+      col16.resize((size_t)D->nnz);
+      for (int64_t e = 0; e < D->nnz; ++e) col16[e] = (uint16_t)c[e];
+    }
+  }
+
+  // ---- upload
+  vqlin_handle* h = new vqlin_handle();
+  memset(h, 0, sizeof *h);
+  cudaGetDevice(&h->device);
+  Uploader up{h};
+  Layer& L = h->L;
+  L.n_out = D->n_out; L.n_in = D->n_in; L.d = d;
+  L.k1 = D->k1; L.bits1 = D->bits1; L.k2 = D->k2; L.bits2 = D->bits2; L.w = w;
+  L.n_main = n_main; L.n_sub = n_sub;
+  L.n_ocols = D->n_ocols; L.n_sub_o = n_sub_o; L.ko = D->n_ocols ? D->ko : 0; L.bits_o = D->n_ocols ? D->bits_o : 0;
+  L.stride = stride; L.stride_o = D->n_ocols ? stride_o : 0;
+  L.codes = up.put<uint8_t>(codes_r.data(), codes_r.size());
+  L.codes_o = D->n_ocols ? up.put<uint8_t>(codes_o_r.data(), codes_o_r.size()) : nullptr;
+  L.cb1 = up.put<__half>(cb1.data(), cb1.size());
+  L.cb2 = D->k2 ? up.put<__half>(cb2.data(), cb2.size()) : nullptr;
+  L.cbo = D->n_ocols ? up.put<__half>(cbo.data(), cbo.size()) : nullptr;
+  L.rs = D->row_scale ? up.put<__half>(rs.data(), rs.size()) : nullptr;
+  L.cs = D->col_scale ? up.put<__half>(cs.data(), cs.size()) : nullptr;
+  L.colmap = D->n_ocols ? up.put<int32_t>(colmap.data(), colmap.size() * 4) : nullptr;
+  L.nnz = D->nnz;
+  if (D->nnz) {
+    L.row_ptr = up.put<int32_t>(rp.data(), rp.size());
+    L.col = up.put<int32_t>(ci.data(), ci.size());
+    L.val = up.put<uint16_t>(vals.data(), vals.size());
+    L.delta = up.put<float>(delta.data(), delta.size() * 4);
+    L.col16 = col16.empty() ? nullptr : up.put<uint16_t>(col16.data(), col16.size() * 2);
+  }
+  if (up.st == VQLIN_OK) up.st = cuda_status(cudaStreamSynchronize((cudaStream_t)stream), "create sync");
+  if (up.st != VQLIN_OK) {
+    vqlin_status s = up.st;
+    vqlin_destroy(h);
+    return s;
+  }
+  // ---- info
+  vqlin_info& I = h->info;
+  I.n_out = D->n_out; I.n_in = D->n_in; I.d = d; I.n_sub = n_sub; I.n_sub_o = n_sub_o; I.n_ocols = D->n_ocols;
+  I.nnz = D->nnz;
+  I.index_bytes = row_bytes * D->n_out + (D->n_ocols ? row_bytes_o * D->n_out : 0);
+  I.codebook_bytes = 2ll * d * (D->k1 + D->k2 + (D->n_ocols ? D->ko : 0));
+  I.scale_bytes = (D->row_scale ? 2ll * D->n_out : 0) + (D->col_scale ? 2ll * D->n_in : 0);
+  I.sparse_bytes = D->nnz ? D->nnz * 6 + 4ll * (D->n_out + 1) : 0;
+  {
+    // VPTQ "Compression ratio calculation": 16*M / (V*k*16 + M*ceil(log2 k)/V)
+    double M = (double)D->n_out * D->n_in;
+    int lb = 0;
+    while ((1ll << lb) < D->k1) ++lb;
+    double ratio = 16.0 * M / ((double)d * D->k1 * 16.0 + M * lb / d);
+    I.vptq_compression_ratio = ratio;
+    I.vptq_bits_per_weight = 16.0 / ratio;
+    double total_bits = 8.0 * (I.index_bytes + I.codebook_bytes + I.scale_bytes + I.sparse_bytes + 4ll * D->n_ocols);
+    I.total_bits_per_weight = total_bits / M;
+  }
+  cudaSetDevice(prev_dev);
+  *out = h;
+  return VQLIN_OK;
+}
+
+vqlin_status vqlin_get_info(const vqlin_handle* h, vqlin_info* info) {
+  if (!h || !info) { set_error("NULL argument"); return VQLIN_ERR_INVALID_ARG; }
+  *info = h->info;
+  return VQLIN_OK;
+}
+
+static bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+vqlin_status vqlin_unpack_indices(const vqlin_handle* h, int32_t which, uint32_t* out, void* stream) {
+  if (!h || !out || (which != 0 && which != 1)) { set_error("bad argument"); return VQLIN_ERR_INVALID_ARG; }
+  if (which == 1 && h->L.n_ocols == 0) return VQLIN_OK;
+  return cuda_status(launch_unpack(h->L, which, out, (cudaStream_t)stream), "unpack launch");
+}
+
+vqlin_status vqlin_dequant(const vqlin_handle* h, uint16_t* W, int64_t ldw, void* stream) {
+  if (!h || !W || ldw < h->L.n_in) { set_error("bad argument (W NULL or ldw < n_in)"); return VQLIN_ERR_INVALID_ARG; }
+  if (!aligned(W, 2)) { set_error("W must be 2-byte aligned"); return VQLIN_ERR_INVALID_ARG; }
+  return cuda_status(launch_dequant(h->L, reinterpret_cast<__half*>(W), ldw, (cudaStream_t)stream), "dequant launch");
+}
+
+static bool dtype_ok(vqlin_dtype t) { return t == VQLIN_F32 || t == VQLIN_F16 || t == VQLIN_BF16; }
+
+vqlin_status vqlin_gemv(const vqlin_handle* h, const void* x, vqlin_dtype xt, int32_t batch, void* y,
+                        vqlin_dtype yt, void* stream) {
+  if (!h || !x || !y) { set_error("NULL argument"); return VQLIN_ERR_INVALID_ARG; }
+  if (!dtype_ok(xt) || !dtype_ok(yt)) { set_error("bad dtype"); return VQLIN_ERR_INVALID_ARG; }
+  if (batch < 1 || batch > VQLIN_MAX_BATCH) { set_error("batch = %d: must be 1..16", batch); return VQLIN_ERR_UNSUPPORTED; }
+  if (!aligned(x, 16) || !aligned(y, 16)) { set_error("x and y must be 16-byte aligned"); return VQLIN_ERR_INVALID_ARG; }
+  return cuda_status(launch_gemv(h->L, x, xt, batch, y, yt, (cudaStream_t)stream), "gemv launch");
+}
+
+static size_t ws_align(size_t b) { return (b + 255) & ~size_t(255); }
+
+size_t vqlin_gemm_workspace_size(const vqlin_handle* h, int64_t M) {
+  if (!h || M < 1) return 0;
+  size_t w = ws_align((size_t)h->L.n_out * h->L.n_in * 2);
+  size_t x = ws_align((size_t)M * h->L.n_in * 2);
+  return w + x;
+}
+
+vqlin_status vqlin_gemm(const vqlin_handle* h, const void* X, vqlin_dtype xt, int64_t M, void* Y, vqlin_dtype yt,
+                        void* workspace, size_t ws_bytes, void* stream) {
+  if (!h || !X || !Y) { set_error("NULL argument"); return VQLIN_ERR_INVALID_ARG; }
+  if (M < 1) { set_error("M must be >= 1"); return VQLIN_ERR_UNSUPPORTED; }
+  if (xt != VQLIN_F16 && xt != VQLIN_BF16) { set_error("X must be F16 or BF16"); return VQLIN_ERR_UNSUPPORTED; }
+  if (!dtype_ok(yt)) { set_error("bad Y dtype"); return VQLIN_ERR_INVALID_ARG; }
+  if (h->L.n_in % 8 != 0) { set_error("gemm needs n_in %% 8 == 0"); return VQLIN_ERR_UNSUPPORTED; }
+  if (!aligned(X, 16) || !aligned(Y, 16)) { set_error("X and Y must be 16-byte aligned"); return VQLIN_ERR_INVALID_ARG; }
+  size_t need = vqlin_gemm_workspace_size(h, M);
+  if (!workspace || ws_bytes < need || !aligned(workspace, 256)) {
+    set_error("workspace must be >= %zu bytes and 256-byte aligned", need);
+    return VQLIN_ERR_WORKSPACE;
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  __half* W = reinterpret_cast<__half*>(workspace);
+  __half* X16 = reinterpret_cast<__half*>(reinterpret_cast<char*>(workspace) + ws_align((size_t)h->L.n_out * h->L.n_in * 2));
+  vqlin_status st = cuda_status(launch_dequant(h->L, W, h->L.n_in, s), "gemm dequant launch");
+  if (st) return st;
+  const __half* A = reinterpret_cast<const __half*>(X);
+  if (xt == VQLIN_BF16) {
+    st = cuda_status(launch_convert_to_f16(X, xt, M * h->L.n_in, X16, s), "gemm convert launch");
+    if (st) return st;
+    A = X16;
+  }
+  return cuda_status(launch_gemm_f16(A, W, M, h->L.n_out, h->L.n_in, Y, yt, s), "gemm launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,235 @@
+// Fused dequantise + GEMV ("QGemv" on the VPTQ page, "The dequantization
+// interface": dequantisation fused into the decode matvec so the fp16 weight
+// is never written or re-read), with the sparse correction fused into the same
+// pass (SCVQ summary step 4; HAS-VQ abstract).
+//
+//   y[b,i] = r_i * sum_s <C1[i1(i,s)] (+ C2[i2(i,s)]), x'[b, s*d : s*d+d]>
+//          + r_i * sum_s' <Co[io(i,s')], x'_o[b, s'*d : s'*d+d]>
+//          + sum_{e in row i} delta_e * x[b, col_e],      x' = c (.) x,
+//
+// where delta_e = v_e - (decoded value at that position) is prepared at create
+// time, so the sparse entries replace the decoded weight exactly (up to the
+// fp32 products).  All products and sums are fp32.
+#include "vqlin_internal.cuh"
+
+namespace vqlin {
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <int D>
+__device__ __forceinline__ void load_centroid(const __half* base, uint32_t idx, float* c) {
+  if (D == 8) {
+    uint4 u = __ldg(reinterpret_cast<const uint4*>(base) + idx);
+    const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) { float2 f = __half22float2(h[k]); c[2 * k] = f.x; c[2 * k + 1] = f.y; }
+  } else {
+    uint2 u = __ldg(reinterpret_cast<const uint2*>(base) + idx);
+    const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) { float2 f = __half22float2(h[k]); c[2 * k] = f.x; c[2 * k + 1] = f.y; }
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void load_centroid_smem(const __half* base, uint32_t idx, float* c) {
+  if (D == 8) {
+    uint4 u = reinterpret_cast<const uint4*>(base)[idx];
+    const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) { float2 f = __half22float2(h[k]); c[2 * k] = f.x; c[2 * k + 1] = f.y; }
+  } else {
+    uint2 u = reinterpret_cast<const uint2*>(base)[idx];
+    const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) { float2 f = __half22float2(h[k]); c[2 * k] = f.x; c[2 * k + 1] = f.y; }
+  }
+}
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kRPW = 2;                 // rows per warp
+constexpr int kRowsPerCta = kWarps * kRPW;
+
+// Generic kernel: any field width <= 32, d in {4, 8}, residual and outlier
+// blocks, batch <= NB.  x' is staged through shared memory in column chunks.
+template <int D, int NB, bool CB_SMEM>
+__global__ void __launch_bounds__(kThreads) k_gemv_generic(Layer L, const void* __restrict__ x, vqlin_dtype xt,
+                                                           int batch, void* __restrict__ y, vqlin_dtype yt,
+                                                           int chunk) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  float* xs = reinterpret_cast<float*>(smem);                       // [NB][chunk]
+  __half* cb1s = reinterpret_cast<__half*>(xs + NB * chunk);
+  __half* cb2s = cb1s + (size_t)L.k1 * D;
+  __half* cbos = cb2s + (size_t)L.k2 * D;
+  const __half* cb1 = L.cb1;
+  const __half* cb2 = L.cb2;
+  const __half* cbo = L.cbo;
+  if (CB_SMEM) {
+    const int n16 = ((L.k1 + L.k2 + L.ko) * D * 2) / 16;   // all three are whole multiples of 8 bytes
+    const uint4* srcs[3] = {reinterpret_cast<const uint4*>(L.cb1), reinterpret_cast<const uint4*>(L.cb2),
+                            reinterpret_cast<const uint4*>(L.cbo)};
+    int lens[3] = {L.k1 * D * 2, L.k2 * D * 2, L.ko * D * 2};
+    unsigned char* dst = reinterpret_cast<unsigned char*>(cb1s);
+    for (int part = 0; part < 3; ++part) {
+      // copy in 8-byte units (d = 4 entries are 8 bytes)
+      const uint2* s2 = reinterpret_cast<const uint2*>(srcs[part]);
+      uint2* d2 = reinterpret_cast<uint2*>(dst);
+      for (int t = threadIdx.x; t < lens[part] / 8; t += kThreads) d2[t] = __ldg(s2 + t);
+      dst += lens[part];
+    }
+    (void)n16;
+    cb1 = cb1s; cb2 = L.cb2 ? cb2s : nullptr; cbo = cbos;
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row0 = blockIdx.x * kRowsPerCta + warp * kRPW;
+  const uint32_t m1 = (1u << L.bits1) - 1u;
+  float acc[kRPW][NB];
+#pragma unroll
+  for (int r = 0; r < kRPW; ++r)
+#pragma unroll
+    for (int b = 0; b < NB; ++b) acc[r][b] = 0.f;
+
+  auto stage = [&](int col_base, int ncols, bool outlier) {
+    __syncthreads();
+    for (int t = threadIdx.x; t < NB * chunk; t += kThreads) {
+      int b = t / chunk, q = t - b * chunk;
+      float v = 0.f;
+      if (b < batch && q < ncols) {
+        int qq = col_base + q;
+        int j = outlier ? L.colmap[L.n_main + qq] : (L.colmap ? L.colmap[qq] : qq);
+        v = load_as_float(x, xt, (int64_t)b * L.n_in + j);
+        if (L.cs) v *= __half2float(L.cs[j]);
+      }
+      xs[t] = v;
+    }
+    __syncthreads();
+  };
+
+  for (int q0 = 0; q0 < L.n_main; q0 += chunk) {
+    const int qn = min(chunk, L.n_main - q0);
+    stage(q0, qn, false);
+    const int s0 = q0 / D, s1 = s0 + (qn + D - 1) / D;
+#pragma unroll
+    for (int r = 0; r < kRPW; ++r) {
+      const int row = row0 + r;
+      if (row >= L.n_out) break;
+      const uint8_t* rowp = L.codes + (int64_t)row * L.stride;
+      for (int s = s0 + lane; s < s1; s += 32) {
+        uint32_t f = read_field(rowp, s, L.w);
+        float c[D];
+        if (CB_SMEM) load_centroid_smem<D>(cb1, f & m1, c); else load_centroid<D>(cb1, f & m1, c);
+        if (cb2) {
+          float c2[D];
+          if (CB_SMEM) load_centroid_smem<D>(cb2, f >> L.bits1, c2); else load_centroid<D>(cb2, f >> L.bits1, c2);
+#pragma unroll
+          for (int k = 0; k < D; ++k) c[k] += c2[k];
+        }
+        const float* xv = xs + (s - s0) * D;
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          float a = acc[r][b];
+#pragma unroll
+          for (int k = 0; k < D; ++k) a = fmaf(c[k], xv[b * chunk + k], a);
+          acc[r][b] = a;
+        }
+      }
+    }
+  }
+  if (L.n_ocols > 0) {
+    stage(0, L.n_ocols, true);
+#pragma unroll
+    for (int r = 0; r < kRPW; ++r) {
+      const int row = row0 + r;
+      if (row >= L.n_out) break;
+      const uint8_t* rowp = L.codes_o + (int64_t)row * L.stride_o;
+      for (int s = lane; s < L.n_sub_o; s += 32) {
+        uint32_t f = read_field(rowp, s, L.bits_o);
+        float c[D];
+        if (CB_SMEM) load_centroid_smem<D>(cbo, f, c); else load_centroid<D>(cbo, f, c);
+        const float* xv = xs + s * D;
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          float a = acc[r][b];
+#pragma unroll
+          for (int k = 0; k < D; ++k) a = fmaf(c[k], xv[b * chunk + k], a);
+          acc[r][b] = a;
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < kRPW; ++r) {
+    const int row = row0 + r;
+    if (row >= L.n_out) break;
+    float sp[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) sp[b] = 0.f;
+    if (L.nnz > 0) {
+      for (int e = L.row_ptr[row] + lane; e < L.row_ptr[row + 1]; e += 32) {
+        const float dl = L.delta[e];
+        const int j = L.col[e];
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+          if (b < batch) sp[b] = fmaf(dl, load_as_float(x, xt, (int64_t)b * L.n_in + j), sp[b]);
+      }
+    }
+    const float rsc = L.rs ? __half2float(L.rs[row]) : 1.f;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      float body = warp_sum(acc[r][b]);
+      float spb = warp_sum(sp[b]);
+      if (lane == 0 && b < batch) store_from_float(y, yt, (int64_t)b * L.n_out + row, fmaf(rsc, body, spb));
+    }
+  }
+}
+
+template <int D, int NB>
+static cudaError_t launch_generic_nb(const Layer& L, const void* x, vqlin_dtype xt, int batch, void* y,
+                                     vqlin_dtype yt, cudaStream_t s) {
+  // x' chunk: at most 48 KB, a multiple of 32*D columns, at least the outlier block
+  int chunk = (48 * 1024) / (4 * NB);
+  chunk = (chunk / (32 * D)) * (32 * D);
+  int need = ((L.n_main + D - 1) / D) * D;
+  if (need < chunk) chunk = ((need + 32 * D - 1) / (32 * D)) * (32 * D);
+  int need_o = L.n_sub_o * D;
+  if (need_o > chunk) chunk = ((need_o + 32 * D - 1) / (32 * D)) * (32 * D);
+  size_t xs_bytes = (size_t)NB * chunk * 4;
+  size_t cb_bytes = (size_t)(L.k1 + L.k2 + L.ko) * D * 2;
+  bool cb_smem = xs_bytes + cb_bytes <= 200 * 1024;
+  size_t smem = xs_bytes + (cb_smem ? cb_bytes : 0);
+  dim3 grid((L.n_out + kRowsPerCta - 1) / kRowsPerCta);
+  if (cb_smem) {
+    auto k = k_gemv_generic<D, NB, true>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k<<<grid, kThreads, smem, s>>>(L, x, xt, batch, y, yt, chunk);
+  } else {
+    auto k = k_gemv_generic<D, NB, false>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k<<<grid, kThreads, smem, s>>>(L, x, xt, batch, y, yt, chunk);
+  }
+  return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_generic(const Layer& L, const void* x, vqlin_dtype xt, int batch, void* y,
+                                  vqlin_dtype yt, cudaStream_t s) {
+  if (batch <= 1) return launch_generic_nb<D, 1>(L, x, xt, batch, y, yt, s);
+  if (batch <= 2) return launch_generic_nb<D, 2>(L, x, xt, batch, y, yt, s);
+  if (batch <= 4) return launch_generic_nb<D, 4>(L, x, xt, batch, y, yt, s);
+  if (batch <= 8) return launch_generic_nb<D, 8>(L, x, xt, batch, y, yt, s);
+  return launch_generic_nb<D, 16>(L, x, xt, batch, y, yt, s);
+}
+
+cudaError_t launch_gemv(const Layer& L, const void* x, vqlin_dtype xt, int batch, void* y, vqlin_dtype yt,
+                        cudaStream_t s) {
+  return L.d == 8 ? launch_generic<8>(L, x, xt, batch, y, yt, s) : launch_generic<4>(L, x, xt, batch, y, yt, s);
+}
+
+}  // namespace vqlin

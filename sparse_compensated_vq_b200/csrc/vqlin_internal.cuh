@@ -1,0 +1,92 @@
+// Internal definitions of libvqlin (device buffer layout of a handle, kernel
+// launchers).  Not part of the public ABI (include/vqlin.h).
+#pragma once
+
+#include <cstdint>
+#include <cstddef>
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+
+#include "vqlin.h"
+
+namespace vqlin {
+
+// Everything a kernel needs to decode a layer.  Device pointers; the handle
+// owns them.  Rows of `codes` / `codes_o` are re-laid out at a 16-byte stride.
+struct Layer {
+  int32_t n_out, n_in, d;
+  int32_t k1, bits1, k2, bits2, w;      // w = bits1 + bits2 (field width)
+  int32_t n_main, n_sub;                // main columns, main sub-vectors per row
+  int32_t n_ocols, n_sub_o, ko, bits_o;
+  int64_t stride, stride_o;             // bytes, multiples of 16
+  const uint8_t* codes;                 // [n_out][stride]
+  const uint8_t* codes_o;               // [n_out][stride_o] or null
+  const __half* cb1;                    // [k1][d]
+  const __half* cb2;                    // [k2][d] or null
+  const __half* cbo;                    // [ko][d] or null
+  const __half* rs;                     // [n_out] or null (= 1)
+  const __half* cs;                     // [n_in]  or null (= 1)
+  const int32_t* colmap;                // [n_in]: main column ids (q order) then outlier ids (p order); null if no outliers
+  int64_t nnz;
+  const int32_t* row_ptr;               // [n_out+1] (null if nnz == 0)
+  const int32_t* col;                   // [nnz]
+  const uint16_t* val;                  // [nnz] fp16 bits (exact replacement values)
+  const float* delta;                   // [nnz] v - body, for the fused products
+  const uint16_t* col16;                // [nnz] column ids as u16 when n_in <= 65536, else null
+};
+
+// Last-error plumbing (thread-local detail string).
+void set_error(const char* fmt, ...);
+vqlin_status cuda_status(cudaError_t e, const char* what);
+
+// Kernel launchers (return cudaGetLastError() of the launch).
+cudaError_t launch_unpack(const Layer& L, int which, uint32_t* out, cudaStream_t s);
+cudaError_t launch_dequant(const Layer& L, __half* W, int64_t ldw, cudaStream_t s);
+cudaError_t launch_gemv(const Layer& L, const void* x, vqlin_dtype xt, int batch, void* y, vqlin_dtype yt,
+                        cudaStream_t s);
+cudaError_t launch_convert_to_f16(const void* X, vqlin_dtype xt, int64_t n, __half* out, cudaStream_t s);
+cudaError_t launch_gemm_f16(const __half* A, const __half* W, int64_t M, int N, int K, void* Y, vqlin_dtype yt,
+                            cudaStream_t s);
+
+// ---- small device helpers shared by the library's kernels -----------------
+__device__ __forceinline__ float load_as_float(const void* p, vqlin_dtype t, int64_t i) {
+  if (t == VQLIN_F32) return __ldg(reinterpret_cast<const float*>(p) + i);
+  unsigned short h = __ldg(reinterpret_cast<const unsigned short*>(p) + i);
+  if (t == VQLIN_F16) return __half2float(__ushort_as_half(h));
+  return __bfloat162float(__ushort_as_bfloat16(h));
+}
+
+__device__ __forceinline__ void store_from_float(void* p, vqlin_dtype t, int64_t i, float v) {
+  if (t == VQLIN_F32) reinterpret_cast<float*>(p)[i] = v;
+  else if (t == VQLIN_F16) reinterpret_cast<__half*>(p)[i] = __float2half_rn(v);
+  else reinterpret_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(v);
+}
+
+// Field s (width w <= 32) of a packed row whose base is 16-byte aligned and whose
+// buffer extends at least 8 bytes past the last field's byte (guaranteed by the
+// 16-byte row stride plus an 16-byte tail pad on the buffer).
+__device__ __forceinline__ uint32_t read_field(const uint8_t* row, int64_t s, int w) {
+  int64_t bit = s * (int64_t)w;
+  const uint8_t* p = row + (bit >> 3);
+  uintptr_t a = reinterpret_cast<uintptr_t>(p);
+  const uint32_t* q = reinterpret_cast<const uint32_t*>(a & ~uintptr_t(3));
+  uint64_t lo = __ldg(q), hi = __ldg(q + 1);
+  uint64_t v = lo | (hi << 32);
+  int sh = int((a & 3) * 8 + (bit & 7));
+  v >>= sh;
+  return w >= 32 ? (uint32_t)v : (uint32_t)(v & ((1ull << w) - 1ull));
+}
+
+}  // namespace vqlin
+
+// The public handle.
+struct vqlin_handle {
+  vqlin::Layer L;
+  int device;
+  // info
+  vqlin_info info;
+  // allocations to free
+  void* allocs[16];
+  int n_allocs;
+};
