@@ -209,6 +209,15 @@ size_t vqlin_gemm_workspace_size(const vqlin_handle* h, int64_t M);
  */
 vqlin_status vqlin_unpack_indices(const vqlin_handle* h, int32_t which, uint32_t* out, void* stream);
 
+/*
+ * Device-side failure detection.  Kernels that wait on hardware barriers bound
+ * every wait (1 s); when one gives up it records a code, skips its remaining
+ * work and returns, so the context stays usable.  This call synchronises the
+ * current device, returns the recorded code in *code (0 = none; 1-5 = the
+ * GEMM pipeline wait that expired) and clears it.  No counterpart on the pages.
+ */
+vqlin_status vqlin_device_error(int32_t* code);
+
 const char* vqlin_status_string(vqlin_status s);
 const char* vqlin_last_error(void);
 int32_t vqlin_abi_version(void);

@@ -104,6 +104,16 @@ const char* vqlin_status_string(vqlin_status s) {
 }
 
 const char* vqlin_last_error(void) { return g_err.c_str(); }
+
+vqlin_status vqlin_device_error(int32_t* code) {
+  if (!code) { set_error("code is NULL"); return VQLIN_ERR_INVALID_ARG; }
+  vqlin_status st = cuda_status(cudaDeviceSynchronize(), "device synchronize");
+  if (st) return st;
+  int v = read_and_clear_device_error();
+  if (v < 0) { set_error("cannot read the device error word"); return VQLIN_ERR_CUDA; }
+  *code = v;
+  return VQLIN_OK;
+}
 int32_t vqlin_abi_version(void) { return VQLIN_ABI_VERSION; }
 
 vqlin_status vqlin_destroy(vqlin_handle* h) {

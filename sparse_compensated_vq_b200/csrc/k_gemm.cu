@@ -1,57 +1,317 @@
-// Prefill GEMM: Y[M][N] = A[M][K] * W[N][K]^T, fp16 operands, fp32 accumulate.
-// (VPTQ page, "The dequantization interface": dequantisation feeds the prefill
-// GEMM.)  The weight operand is the exact fp16 dequantised weight.
+// Prefill GEMM on the 5th-generation tensor cores:
+//   Y[M][N] = A[M][K] * W[N][K]^T,  A = fp16 activations, W = the exact fp16
+//   dequantised weight (VPTQ page, "The dequantization interface": the
+//   dequantised weight feeds the prefill GEMM), fp32 accumulation in TMEM.
+//
+// One CTA computes a 128 x 256 tile of Y:
+//   warp 0      TMA producer: A and W K-blocks (64 fp16 = one 128-byte swizzle
+//               row) into a 4-stage shared-memory ring, completion on mbarriers;
+//   warp 1      allocates 256 TMEM columns and, from one lane, issues
+//               tcgen05.mma.kind::f16 (M=128, N=256, K=16) per K-step, returning
+//               each ring slot with tcgen05.commit;
+//   warps 2-5   epilogue: tcgen05.ld of their 32-lane TMEM quadrant, convert, store.
+// Every mbarrier wait is bounded (1 s of %globaltimer): on expiry the kernel
+// records an error code in vqlin_device_error, stops issuing work, waits (again
+// bounded) for its own copies in flight, frees TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "vqlin_internal.cuh"
 
 namespace vqlin {
 
-// Straightforward shared-memory tiled kernel: 64x64 output tile, 256 threads,
-// 4x4 outputs per thread.
-__global__ void __launch_bounds__(256) k_gemm_simt(const __half* __restrict__ A, const __half* __restrict__ W,
-                                                   int64_t M, int N, int K, void* __restrict__ Y,
-                                                   vqlin_dtype yt) {
-  __shared__ float As[16][64 + 1];
-  __shared__ float Ws[16][64 + 1];
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  const int64_t m0 = (int64_t)blockIdx.y * 64;
-  const int n0 = blockIdx.x * 64;
-  float acc[4][4] = {};
-  for (int k0 = 0; k0 < K; k0 += 16) {
-    for (int t = threadIdx.x; t < 16 * 64; t += 256) {
-      int r = t / 16, kk = t % 16;
-      int64_t m = m0 + r;
-      int n = n0 + r;
-      As[kk][r] = (m < M && k0 + kk < K) ? __half2float(A[m * K + k0 + kk]) : 0.f;
-      Ws[kk][r] = (n < N && k0 + kk < K) ? __half2float(W[(int64_t)n * K + k0 + kk]) : 0.f;
+__device__ int g_device_error = 0;
+
+namespace tc {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;       // 16 KB
+constexpr int B_BYTES = BN * BK * 2;       // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int THREADS = 192;
+constexpr int TMEM_COLS = 256;
+constexpr unsigned long long WAIT_NS = 1000000000ull;   // 1 s
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+
+__device__ __forceinline__ uint64_t now_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait; false on timeout (and records the error).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int code) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = now_ns();
+  while (!mbar_try(bar, parity)) {
+    if (now_ns() - t0 > WAIT_NS) {
+      atomicExch(&g_device_error, code);
+      return false;
     }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < 16; ++kk) {
-      float a[4], b[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) { a[i] = As[kk][ty * 4 + i]; b[i] = Ws[kk][tx * 4 + i]; }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
-    }
-    __syncthreads();
   }
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      int64_t m = m0 + ty * 4 + i;
-      int n = n0 + tx * 4 + j;
-      if (m < M && n < N) store_from_float(Y, yt, m * N + n, acc[i][j]);
+  return true;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+
+// Shared-memory matrix descriptor, K-major operand in the 128-byte swizzle
+// layout: 8-row atoms of 8 x 128 B, atoms 1024 B apart (stride byte offset);
+// the leading byte offset is not used by this layout; version 1; layout 2.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
+}
+
+// Instruction descriptor, kind::f16: D = f32 (bits 4-5 = 1), A = B = f16
+// (bits 7-9, 10-12 = 0), both K-major (bits 15, 16 = 0), N >> 3 at bits 17-22,
+// M >> 4 at bits 24-28.
+__host__ __device__ constexpr uint32_t idesc_f16(int m, int n) {
+  return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}"
+      ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_w, int64_t M,
+              int N, int K, void* __restrict__ Y, vqlin_dtype yt) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // 1024-byte aligned ring (the 128-byte swizzle atoms need it)
+  unsigned char* ring = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + (size_t)STAGES * STAGE_BYTES);
+  // bars[0..S): full, bars[S..2S): empty, bars[2S]: accumulator ready
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t m0 = (int64_t)blockIdx.y * BM;
+  const int n0 = blockIdx.x * BN;
+  const int num_kb = (K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&bars[s]), 1);
+      mbar_init(smem_u32(&bars[STAGES + s]), 1);
     }
+    mbar_init(smem_u32(&bars[2 * STAGES]), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_a)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_w)) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = *tmem_holder;
+  int issued = 0;   // producer: K-blocks whose copies were issued
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer
+    for (int kb = 0; kb < num_kb; ++kb) {
+      const int s = kb % STAGES;
+      const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
+      if (*abort_flag || !mbar_wait(smem_u32(&bars[STAGES + s]), ph ^ 1u, 1)) { *abort_flag = 1; break; }
+      const uint32_t full = smem_u32(&bars[s]);
+      mbar_expect_tx(full, STAGE_BYTES);
+      unsigned char* a = ring + (size_t)s * STAGE_BYTES;
+      tma_load_2d(smem_u32(a), &map_a, full, kb * BK, (int)m0);
+      tma_load_2d(smem_u32(a + A_BYTES), &map_w, full, kb * BK, n0);
+      issued = kb + 1;
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    constexpr uint32_t idesc = idesc_f16(BM, BN);
+    for (int kb = 0; kb < num_kb; ++kb) {
+      const int s = kb % STAGES;
+      const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
+      if (*abort_flag || !mbar_wait(smem_u32(&bars[s]), ph, 2)) { *abort_flag = 1; break; }
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t a = smem_u32(ring + (size_t)s * STAGE_BYTES);
+      const uint64_t da = desc_sw128(a), db = desc_sw128(a + A_BYTES);
+#pragma unroll
+      for (int k = 0; k < BK / 16; ++k)   // 16 fp16 = 32 bytes per step along K inside the swizzle row
+        mma_f16(tmem, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), idesc, (kb | k) != 0);
+      mma_commit(smem_u32(&bars[STAGES + s]));
+    }
+    mma_commit(smem_u32(&bars[2 * STAGES]));
+  } else if (warp >= 2) {
+    // ---------------- epilogue
+    const int q = warp & 3;                        // TMEM lane quadrant this warp may access
+    const int64_t row = m0 + q * 32 + lane;
+    bool ok = mbar_wait(smem_u32(&bars[2 * STAGES]), 0, 3);
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    if (ok && !*abort_flag) {
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c, r);
+        if (row < M) {
+          const int nb = n0 + c;
+          if (yt == VQLIN_F32) {
+            float* yp = reinterpret_cast<float*>(Y) + row * N + nb;
+            if (nb + 32 <= N && (N % 4) == 0) {
+#pragma unroll
+              for (int j = 0; j < 32; j += 4)
+                *reinterpret_cast<float4*>(yp + j) = make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
+                                                                 __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+            } else {
+              for (int j = 0; j < 32; ++j) if (nb + j < N) yp[j] = __uint_as_float(r[j]);
+            }
+          } else {
+            uint32_t packed[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              float lo = __uint_as_float(r[2 * j]), hi = __uint_as_float(r[2 * j + 1]);
+              if (yt == VQLIN_F16) {
+                __half2 h = __floats2half2_rn(lo, hi);
+                packed[j] = *reinterpret_cast<uint32_t*>(&h);
+              } else {
+                __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+                packed[j] = *reinterpret_cast<uint32_t*>(&h);
+              }
+            }
+            unsigned short* yp = reinterpret_cast<unsigned short*>(Y) + row * N + nb;
+            if (nb + 32 <= N && (N % 8) == 0) {
+#pragma unroll
+              for (int j = 0; j < 16; j += 4)
+                *reinterpret_cast<uint4*>(yp + 2 * j) = make_uint4(packed[j], packed[j + 1], packed[j + 2], packed[j + 3]);
+            } else {
+              for (int j = 0; j < 32; ++j)
+                if (nb + j < N) yp[j] = (unsigned short)((packed[j >> 1] >> (16 * (j & 1))) & 0xFFFFu);
+            }
+          }
+        }
+      }
+    }
+  }
+  // ---------------- teardown
+  if (warp == 0 && lane == 0 && *abort_flag) {
+    // let the copies this CTA issued land before its shared memory goes away
+    for (int kb = (issued > STAGES ? issued - STAGES : 0); kb < issued; ++kb)
+      mbar_wait(smem_u32(&bars[kb % STAGES]), (uint32_t)(kb / STAGES) & 1u, 4);
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 1) {
+    // the MMAs must have finished with TMEM before it is released (the final
+    // commit covers every MMA this CTA issued; a no-op wait on the normal path)
+    if (lane == 0) mbar_wait(smem_u32(&bars[2 * STAGES]), 0, 5);
+    __syncwarp();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+  }
+}
+
+}  // namespace tc
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// Row-major [rows][cols] fp16 matrix as a 2-D tensor map with a box of
+// box_rows x 64 columns, 128-byte swizzle, zero fill out of bounds.
+static bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
 }
 
 cudaError_t launch_gemm_f16(const __half* A, const __half* W, int64_t M, int N, int K, void* Y, vqlin_dtype yt,
                             cudaStream_t s) {
-  dim3 grid((N + 63) / 64, (unsigned)((M + 63) / 64));
-  k_gemm_simt<<<grid, 256, 0, s>>>(A, W, M, N, K, Y, yt);
+  // TMA needs 16-byte aligned bases and row strides (K % 8 == 0, checked by the caller)
+  if ((reinterpret_cast<uintptr_t>(A) & 15) || (reinterpret_cast<uintptr_t>(W) & 15) || (K % 8) || M > 0x7FFFFFFF)
+    return cudaErrorInvalidValue;
+  CUtensorMap ma, mw;
+  if (!make_map(&ma, A, (uint64_t)M, (uint64_t)K, tc::BM) || !make_map(&mw, W, (uint64_t)N, (uint64_t)K, tc::BN))
+    return cudaErrorInvalidValue;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(tc::k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  dim3 grid((N + tc::BN - 1) / tc::BN, (unsigned)((M + tc::BM - 1) / tc::BM));
+  tc::k_gemm_tc<<<grid, tc::THREADS, tc::SMEM_BYTES, s>>>(ma, mw, M, N, K, Y, yt);
   return cudaGetLastError();
+}
+
+int read_and_clear_device_error() {
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof v) != cudaSuccess) return -1;
+  if (v) cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero);
+  return v;
 }
 
 }  // namespace vqlin

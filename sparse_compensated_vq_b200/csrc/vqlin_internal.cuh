@@ -46,6 +46,7 @@ cudaError_t launch_dequant(const Layer& L, __half* W, int64_t ldw, cudaStream_t 
 cudaError_t launch_gemv(const Layer& L, const void* x, vqlin_dtype xt, int batch, void* y, vqlin_dtype yt,
                         cudaStream_t s);
 cudaError_t launch_convert_to_f16(const void* X, vqlin_dtype xt, int64_t n, __half* out, cudaStream_t s);
+int read_and_clear_device_error();
 cudaError_t launch_gemm_f16(const __half* A, const __half* W, int64_t M, int N, int K, void* Y, vqlin_dtype yt,
                             cudaStream_t s);
 

@@ -80,10 +80,18 @@ vqlin_unpack_indices = _sig("vqlin_unpack_indices", _S, [_H, C.c_int32, _P, _P])
 vqlin_status_string = _sig("vqlin_status_string", C.c_char_p, [_S])
 vqlin_last_error = _sig("vqlin_last_error", C.c_char_p, [])
 vqlin_abi_version = _sig("vqlin_abi_version", C.c_int32, [])
+vqlin_device_error = _sig("vqlin_device_error", _S, [C.POINTER(C.c_int32)])
 
 EXPORTS = ["vqlin_create", "vqlin_destroy", "vqlin_get_info", "vqlin_dequant", "vqlin_gemv", "vqlin_gemm",
            "vqlin_gemm_workspace_size", "vqlin_unpack_indices", "vqlin_status_string", "vqlin_last_error",
-           "vqlin_abi_version"]
+           "vqlin_abi_version", "vqlin_device_error"]
+
+
+def device_error() -> int:
+    """Synchronise and return (and clear) the code of a kernel that gave up a bounded wait."""
+    c = C.c_int32(0)
+    check(vqlin_device_error(C.byref(c)), "vqlin_device_error")
+    return int(c.value)
 
 
 class VQLinError(RuntimeError):

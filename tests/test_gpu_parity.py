@@ -257,6 +257,7 @@ def run_gemm(vq, L, Xbits, xdt, ydt):
     X = G.torch_x(Xbits, xdt)
     Y = m.gemm(X, out_dtype=G.torch_dtype(ydt))
     torch.cuda.synchronize()
+    assert vq.device_error() == 0, "a GEMM pipeline wait expired"
     return G.to_f64(Y)
 
 
