@@ -197,6 +197,8 @@ def run_vqlin(args, rank, world, dist):
     wl = make_workload(args.config, args.batch)
     wbytes = wl.weight_bytes()
     n_copies = int(min(64, max(1, math.ceil(3 * L2_BYTES / wbytes))))
+    if args.copies:
+        n_copies = args.copies          # 1 = the same weights every step (warm L2), for diagnosis only
     copies = [[vqlin.VQLinear(L) for L in wl.layers] for _ in range(n_copies)]
     xdt = "bf16" if wl.name.startswith(("smollm", "prefill")) else "f16"
     tdt = torch.bfloat16 if xdt == "bf16" else torch.float16
@@ -208,9 +210,11 @@ def run_vqlin(args, rank, world, dist):
 
     xs = [dev_x(wl.xs[li], B) for li, B in wl.calls]
     ys = [torch.empty((B, wl.layers[li].n_out), dtype=tdt, device="cuda") for li, B in wl.calls]
-    ws = None
     if wl.kind == "gemm":
         ws = torch.empty(copies[0][0].workspace_size(wl.calls[0][1]), dtype=torch.uint8, device="cuda")
+    else:   # gemv scratch for column-split accumulation (one buffer reused by every call of the step)
+        need = max(int(vqlin.vqlin_gemv_workspace_size(copies[0][li].handle, B)) for li, B in wl.calls)
+        ws = torch.empty(need, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.Stream()
 
     def step(i, s_handle):
@@ -218,15 +222,16 @@ def run_vqlin(args, rank, world, dist):
         for k, (li, B) in enumerate(wl.calls):
             h = c[li].handle
             if wl.kind == "gemv":
-                st = vqlin.vqlin_gemv(h, xs[k].data_ptr(), vqlin.dtype_code(tdt), B, ys[k].data_ptr(),
-                                      vqlin.dtype_code(tdt), s_handle)
+                st = vqlin.vqlin_gemv_ws(h, xs[k].data_ptr(), vqlin.dtype_code(tdt), B, ys[k].data_ptr(),
+                                         vqlin.dtype_code(tdt), ws.data_ptr(), ws.numel(), s_handle)
             else:
                 st = vqlin.vqlin_gemm(h, xs[k].data_ptr(), vqlin.dtype_code(tdt), B, ys[k].data_ptr(),
                                       vqlin.dtype_code(tdt), ws.data_ptr(), ws.numel(), s_handle)
             if st != 0:
                 raise vqlin.VQLinError(st, "bench step")
 
-    # our kernels per step: one per gemv call; gemm = dequant body + sparse replace + bf16->fp16 + GEMM
+    # our kernels per step: gemv = one kernel per call (+ a finalize kernel when the call splits its
+    # columns, counted below from the plan); gemm = dequant body + sparse replace + bf16->fp16 + GEMM
     launches_per_step = len(wl.calls) if wl.kind == "gemv" else 4
     s_ptr = stream.cuda_stream
     with torch.cuda.stream(stream):
@@ -399,6 +404,7 @@ def main():
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--copies", type=int, default=0, help="override the number of rotating weight copies")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -183,11 +183,26 @@ vqlin_status vqlin_dequant(const vqlin_handle* h, uint16_t* W, int64_t ldw, void
  *   y[b*n_out + i] = sum_j W[i,j] * x[b*n_in + j],  0 <= b < batch <= 16.
  * x: device [batch][n_in] of xt (F16, BF16 or F32); y: device [batch][n_out]
  * of yt.  Products and sums are fp32 (W's unrounded value r*c*C enters through
- * fp32 arithmetic, not through an fp16 weight).  x and y must be 16-byte
- * aligned and must not overlap.  Summation order is unspecified.
+ * fp32 arithmetic, not through an fp16 weight; with d = 8 the tensor-core path
+ * carries x' = c*x as two fp16 parts, so |c_j x_j| must stay below 65504).
+ * x and y must be 16-byte aligned and must not overlap.  Summation order is
+ * unspecified.
  */
 vqlin_status vqlin_gemv(const vqlin_handle* h, const void* x, vqlin_dtype xt, int32_t batch,
                         void* y, vqlin_dtype yt, void* stream);
+
+/*
+ * The same product with a caller-owned scratch buffer: when the layer is too
+ * wide for one pass of the tensor-core decode kernel, column chunks are summed
+ * in fp32 in `workspace` (>= vqlin_gemv_workspace_size(h, batch) bytes, 256-byte
+ * aligned, device memory, not used by another call at the same time) and
+ * converted to yt at the end; vqlin_gemv instead has each thread block loop over
+ * the chunks itself.  Results agree within the GEMV tolerance (summation order
+ * differs).  Errors additionally: WORKSPACE.
+ */
+vqlin_status vqlin_gemv_ws(const vqlin_handle* h, const void* x, vqlin_dtype xt, int32_t batch,
+                           void* y, vqlin_dtype yt, void* workspace, size_t ws_bytes, void* stream);
+size_t vqlin_gemv_workspace_size(const vqlin_handle* h, int32_t batch);
 
 /*
  * Prefill: Y[m*n_out + i] = sum_j W[i,j] * X[m*n_in + j] for 0 <= m < M.

@@ -48,6 +48,12 @@ uint32_t host_field(const uint8_t* row, int64_t s, int w) {
   return w >= 32 ? (uint32_t)v : (uint32_t)(v & ((1ull << w) - 1ull));
 }
 
+void host_put_field(uint8_t* row, int64_t k, int w, uint32_t v) {
+  int64_t bit = k * (int64_t)w;
+  for (int b = 0; b < w; ++b, ++bit)
+    if ((v >> b) & 1u) row[bit >> 3] |= (uint8_t)(1u << (bit & 7));
+}
+
 // Copy `bytes` from a caller buffer (device or host) into a host vector.
 vqlin_status fetch(const void* src, size_t bytes, bool on_host, std::vector<uint8_t>& dst, const char* what) {
   dst.resize(bytes);
@@ -298,6 +304,28 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
     }
   }
 
+  // tensor-core decode layout (see vqlin_internal.cuh)
+  std::vector<uint8_t> tcodes;
+  int32_t n_ls = 0;
+  int64_t tstride = 0;
+  if (d == 8 && n_sub > 0 && (w == 8 || w == 12 || w == 16 || w == 24 || w == 32)) {
+    n_ls = (int32_t)ceil_div(n_sub, 64);
+    tstride = (int64_t)n_ls * 8 * w;
+    const int64_t rows_pad = round_up(D->n_out, 16);
+    tcodes.assign((size_t)(rows_pad * tstride), 0);
+    for (int32_t i = 0; i < D->n_out; ++i) {
+      const uint8_t* row = codes.data() + (size_t)i * D->row_stride_bytes;
+      uint8_t* dst = tcodes.data() + (size_t)i * tstride;
+      for (int32_t ls = 0; ls < n_ls; ++ls)
+        for (int t = 0; t < 4; ++t)
+          for (int ps = 0; ps < 16; ++ps) {
+            int32_t sv = 64 * ls + 4 * ps + t;
+            if (sv >= n_sub) continue;   // padding fields stay 0 (a valid index; x' is 0 there)
+            host_put_field(dst, (int64_t)ls * 64 + t * 16 + ps, w, host_field(row, sv, w));
+          }
+    }
+  }
+
   // ---- upload
   vqlin_handle* h = new vqlin_handle();
   memset(h, 0, sizeof *h);
@@ -325,6 +353,9 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
     L.delta = up.put<float>(delta.data(), delta.size() * 4);
     L.col16 = col16.empty() ? nullptr : up.put<uint16_t>(col16.data(), col16.size() * 2);
   }
+  L.tcodes = tcodes.empty() ? nullptr : up.put<uint8_t>(tcodes.data(), tcodes.size());
+  L.n_ls = n_ls;
+  L.tstride = tstride;
   if (up.st == VQLIN_OK) up.st = cuda_status(cudaStreamSynchronize((cudaStream_t)stream), "create sync");
   if (up.st != VQLIN_OK) {
     vqlin_status s = up.st;
@@ -383,7 +414,26 @@ vqlin_status vqlin_gemv(const vqlin_handle* h, const void* x, vqlin_dtype xt, in
   if (!dtype_ok(xt) || !dtype_ok(yt)) { set_error("bad dtype"); return VQLIN_ERR_INVALID_ARG; }
   if (batch < 1 || batch > VQLIN_MAX_BATCH) { set_error("batch = %d: must be 1..16", batch); return VQLIN_ERR_UNSUPPORTED; }
   if (!aligned(x, 16) || !aligned(y, 16)) { set_error("x and y must be 16-byte aligned"); return VQLIN_ERR_INVALID_ARG; }
-  return cuda_status(launch_gemv(h->L, x, xt, batch, y, yt, (cudaStream_t)stream), "gemv launch");
+  return cuda_status(launch_gemv(h->L, x, xt, batch, y, yt, nullptr, 0, (cudaStream_t)stream), "gemv launch");
+}
+
+size_t vqlin_gemv_workspace_size(const vqlin_handle* h, int32_t batch) {
+  if (!h || batch < 1 || batch > VQLIN_MAX_BATCH) return 0;
+  return gemv_workspace_bytes(h->L, batch);
+}
+
+vqlin_status vqlin_gemv_ws(const vqlin_handle* h, const void* x, vqlin_dtype xt, int32_t batch, void* y,
+                           vqlin_dtype yt, void* workspace, size_t ws_bytes, void* stream) {
+  if (!h || !x || !y) { set_error("NULL argument"); return VQLIN_ERR_INVALID_ARG; }
+  if (!dtype_ok(xt) || !dtype_ok(yt)) { set_error("bad dtype"); return VQLIN_ERR_INVALID_ARG; }
+  if (batch < 1 || batch > VQLIN_MAX_BATCH) { set_error("batch = %d: must be 1..16", batch); return VQLIN_ERR_UNSUPPORTED; }
+  if (!aligned(x, 16) || !aligned(y, 16)) { set_error("x and y must be 16-byte aligned"); return VQLIN_ERR_INVALID_ARG; }
+  if (!workspace || ws_bytes < gemv_workspace_bytes(h->L, batch) || !aligned(workspace, 256)) {
+    set_error("workspace must be >= %zu bytes and 256-byte aligned", gemv_workspace_bytes(h->L, batch));
+    return VQLIN_ERR_WORKSPACE;
+  }
+  return cuda_status(launch_gemv(h->L, x, xt, batch, y, yt, workspace, ws_bytes, (cudaStream_t)stream),
+                     "gemv launch");
 }
 
 static size_t ws_align(size_t b) { return (b + 255) & ~size_t(255); }

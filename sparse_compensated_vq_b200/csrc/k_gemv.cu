@@ -227,9 +227,17 @@ static cudaError_t launch_generic(const Layer& L, const void* x, vqlin_dtype xt,
   return launch_generic_nb<D, 16>(L, x, xt, batch, y, yt, s);
 }
 
-cudaError_t launch_gemv(const Layer& L, const void* x, vqlin_dtype xt, int batch, void* y, vqlin_dtype yt,
-                        cudaStream_t s) {
+cudaError_t launch_gemv_generic(const Layer& L, const void* x, vqlin_dtype xt, int batch, void* y, vqlin_dtype yt,
+                                cudaStream_t s) {
   return L.d == 8 ? launch_generic<8>(L, x, xt, batch, y, yt, s) : launch_generic<4>(L, x, xt, batch, y, yt, s);
+}
+
+cudaError_t launch_gemv(const Layer& L, const void* x, vqlin_dtype xt, int batch, void* y, vqlin_dtype yt,
+                        void* ws, size_t ws_bytes, cudaStream_t s) {
+  bool handled = false;
+  cudaError_t e = launch_gemv_tc(L, x, xt, batch, y, yt, ws, ws_bytes, s, &handled);
+  if (e != cudaSuccess || handled) return e;
+  return launch_gemv_generic(L, x, xt, batch, y, yt, s);
 }
 
 }  // namespace vqlin

@@ -1,0 +1,505 @@
+// Tensor-core decode GEMV (d = 8): the fused dequant + GEMV of the VPTQ page
+// ("The dequantization interface", QGemv) with the gathered centroids as the
+// A operand of mma.sync m16n8k16 and the activations as the B operand.
+//
+//   A[16 rows][16 k]  = fp16 centroids of 16 weight rows (one per sub-vector);
+//                       the scales are not applied to A, so A is exact;
+//   B[16 k][8 n]      = x' = c (.) x split into fp16 hi + lo parts (columns of
+//                       B are (batch, part) pairs), so hi*A + lo*A keeps the
+//                       fp32 product to ~2^-22 relative;
+//   D[16 rows][8 n]   fp32 accumulators; y = r * (D_hi + D_lo) + sparse term.
+//
+// A residual codebook (VPTQ "Residual Vector Quantization": C1[i1] + C2[i2])
+// issues a second MMA with the C2 centroids as A (no fp16 rounding of the sum).
+//
+// Index layout.  At create time the packed fields are re-laid out per row so
+// that the lane that needs them can fetch them with one vector load: for each
+// "layout slab" of 64 sub-vectors and each t in 0..3, the 16 fields of the
+// sub-vectors 64*slab + 4*ps + t (ps = 0..15) are stored consecutively
+// (LSB-first, same width w).  Thread (g, t) of a warp then owns sub-vector t of
+// every group of four, which is exactly the k-range (2t, 2t+1, 2t+8, 2t+9) the
+// m16n8k16 fragments give it once the eight elements of a centroid are mapped
+// to k = {2t, 2t+1} (elements 0,1 / 4,5) and {2t+8, 2t+9} (elements 2,3 / 6,7).
+//
+// Work.  A CTA task is (RTT row tiles of 16 rows) x (a chunk of kernel slabs);
+// each warp owns one (row tile, kernel slab) pair per chunk, keeps that slab's
+// B fragments in registers, and accumulates its D fragment.  Warps of a task
+// are reduced through shared memory and the epilogue adds the fused sparse
+// correction (delta_e * x_j) and the outlier-column block on CUDA cores.  With
+// more columns than one task covers, either the CTA loops over the chunks
+// (no scratch), or tasks are split by chunk and accumulate in fp32 with
+// atomics (caller workspace, or y itself when y is fp32).
+#include "vqlin_internal.cuh"
+
+namespace vqlin {
+
+namespace tcg {
+
+constexpr int WARPS = 8;
+constexpr int THREADS = WARPS * 32;
+
+__device__ __forceinline__ void mma16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Load the fields one kernel slab needs from a (row, layout slab, t) block:
+// 16/NT fields of W bits = 2W/NT bytes, with the widest naturally aligned vector.
+template <int W, int NT>
+__device__ __forceinline__ void load_sub(const uint8_t* p, uint32_t* w) {
+  constexpr int BYTES = 2 * W / NT;
+  constexpr int VW = (BYTES % 16 == 0) ? 16 : (BYTES % 8 == 0) ? 8 : (BYTES % 4 == 0) ? 4 : 2;
+  if constexpr (VW == 16) {
+#pragma unroll
+    for (int i = 0; i < BYTES / 16; ++i) {
+      uint4 v = __ldg(reinterpret_cast<const uint4*>(p) + i);
+      w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+    }
+  } else if constexpr (VW == 8) {
+#pragma unroll
+    for (int i = 0; i < BYTES / 8; ++i) {
+      uint2 v = __ldg(reinterpret_cast<const uint2*>(p) + i);
+      w[2 * i] = v.x; w[2 * i + 1] = v.y;
+    }
+  } else if constexpr (VW == 4) {
+#pragma unroll
+    for (int i = 0; i < BYTES / 4; ++i) w[i] = __ldg(reinterpret_cast<const uint32_t*>(p) + i);
+  } else {
+#pragma unroll
+    for (int i = 0; i < BYTES / 2; ++i) {
+      uint32_t h = __ldg(reinterpret_cast<const unsigned short*>(p) + i);
+      if (i & 1) w[i >> 1] |= h << 16; else w[i >> 1] = h;
+    }
+  }
+}
+
+template <int W>
+__device__ __forceinline__ uint32_t field_of(const uint32_t* w, int k) {
+  const int bit = k * W;
+  if constexpr (W == 8 || W == 16 || W == 32) {
+    return W == 32 ? w[k] : (w[bit >> 5] >> (bit & 31)) & ((1u << W) - 1u);
+  } else {
+    const int lo = bit >> 5, sh = bit & 31;
+    uint32_t v = (sh + W <= 32) ? (w[lo] >> sh) : __funnelshift_r(w[lo], w[lo + 1], sh);
+    return v & ((1u << W) - 1u);
+  }
+}
+
+struct Args {
+  Layer L;
+  const void* x;
+  vqlin_dtype xt;
+  int batch;
+  void* y;
+  vqlin_dtype yt;
+  float* acc;         // split mode: fp32 [batch][n_out] accumulator (may alias y when yt == F32)
+  int split;          // 0: a task covers every chunk; 1: tasks are (row group, chunk)
+  int n_kslabs;       // kernel slabs over the main columns
+  int ks;             // kernel slabs per chunk handled together (<= WARPS)
+  int rtt;            // row tiles per task (WARPS / ks)
+  int n_chunks;       // ceil(n_kslabs / ks)
+  int xs_cols;        // columns of x' held in shared memory (chunk columns, or all)
+  int xs_all;         // 1: x' for all main columns staged once per CTA
+};
+
+template <int NT, int W, bool CB_SMEM, int COPIES>
+__global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
+  constexpr int PS = 16 / NT;            // pair-steps (4 sub-vectors each) per kernel slab
+  constexpr int KSV = 4 * PS;            // sub-vectors per kernel slab
+  constexpr int BP = 4 * NT;             // batch slots
+  const Layer& L = a.L;
+  extern __shared__ __align__(16) unsigned char smem[];
+  // ---- shared memory carve-up
+  unsigned char* sp = smem;
+  uint4* cb1s = reinterpret_cast<uint4*>(sp);
+  uint4* cb2s = cb1s + (CB_SMEM ? (size_t)L.k1 * COPIES : 0);
+  sp = reinterpret_cast<unsigned char*>(cb2s + (CB_SMEM ? (size_t)L.k2 * COPIES : 0));
+  __half* xh = reinterpret_cast<__half*>(sp);                      // [batch][xs_cols]
+  __half* xl = xh + (size_t)a.batch * a.xs_cols;
+  float* red = reinterpret_cast<float*>(xl + (size_t)a.batch * a.xs_cols);   // [rtt][16][8*NT]
+  float* xo = red + (size_t)a.rtt * 16 * 8 * NT;                        // outlier x' [BP][n_sub_o*8]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int B = a.batch;
+  const uint32_t m1 = (1u << L.bits1) - 1u;
+
+  // ---- codebooks into shared memory (COPIES interleaved copies: entry k of copy c at k*COPIES + c)
+  if (CB_SMEM) {
+    const uint4* c1 = reinterpret_cast<const uint4*>(L.cb1);
+    for (int i = threadIdx.x; i < L.k1 * COPIES; i += THREADS) cb1s[i] = __ldg(c1 + i / COPIES);
+    if (L.k2) {
+      const uint4* c2 = reinterpret_cast<const uint4*>(L.cb2);
+      for (int i = threadIdx.x; i < L.k2 * COPIES; i += THREADS) cb2s[i] = __ldg(c2 + i / COPIES);
+    }
+  }
+  // ---- outlier-block x' (fp32), once per CTA
+  const int n_o = L.n_sub_o * 8;
+  for (int i = threadIdx.x; i < BP * n_o; i += THREADS) {
+    int b = i / n_o, p = i - b * n_o;
+    float v = 0.f;
+    if (b < B && p < L.n_ocols) {
+      int j = L.colmap[L.n_main + p];
+      v = load_as_float(a.x, a.xt, (int64_t)b * L.n_in + j);
+      if (L.cs) v *= __half2float(L.cs[j]);
+    }
+    xo[i] = v;
+  }
+
+  // x' = c (.) x for main columns [col0, col0 + ncols) of every batch row, split
+  // into fp16 hi + lo; eight consecutive columns per thread, all loads first.
+  auto stage_x = [&](int col0, int ncols) {
+    const int groups = ncols / 8;
+    for (int i = threadIdx.x; i < B * groups; i += THREADS) {
+      const int b = i / groups, q = (i - b * groups) * 8;
+      const int qq = col0 + q;
+      float v[8];
+      if (!L.colmap && a.xt != VQLIN_F32 && qq + 8 <= L.n_main && (L.n_in & 7) == 0) {
+        uint4 u = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const unsigned short*>(a.x) +
+                                                        (int64_t)b * L.n_in + qq));
+        const unsigned short* hs = reinterpret_cast<const unsigned short*>(&u);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          v[k] = a.xt == VQLIN_F16 ? __half2float(__ushort_as_half(hs[k])) : __bfloat162float(__ushort_as_bfloat16(hs[k]));
+        if (L.cs) {
+          uint4 cu = __ldg(reinterpret_cast<const uint4*>(L.cs + qq));
+          const __half* cv = reinterpret_cast<const __half*>(&cu);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) v[k] *= __half2float(cv[k]);
+        }
+      } else {
+        int jj[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int c = qq + k;
+          jj[k] = c < L.n_main ? (L.colmap ? L.colmap[c] : c) : -1;
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = jj[k] >= 0 ? load_as_float(a.x, a.xt, (int64_t)b * L.n_in + jj[k]) : 0.f;
+        if (L.cs) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) v[k] *= jj[k] >= 0 ? __half2float(L.cs[jj[k]]) : 0.f;
+        }
+      }
+      uint32_t ph[4], pl[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        __half h0 = __float2half_rn(v[2 * k]), h1 = __float2half_rn(v[2 * k + 1]);
+        __half l0 = __float2half_rn(v[2 * k] - __half2float(h0)), l1 = __float2half_rn(v[2 * k + 1] - __half2float(h1));
+        ph[k] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16);
+        pl[k] = (uint32_t)__half_as_ushort(l0) | ((uint32_t)__half_as_ushort(l1) << 16);
+      }
+      *reinterpret_cast<uint4*>(xh + (size_t)b * a.xs_cols + q) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+      *reinterpret_cast<uint4*>(xl + (size_t)b * a.xs_cols + q) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+    }
+  };
+
+  const int n_rt = (L.n_out + 15) / 16;
+  const int n_rg = (n_rt + a.rtt - 1) / a.rtt;
+  const int n_tasks = a.split ? n_rg * a.n_chunks : n_rg;
+  const int chunk_cols = a.ks * KSV * 8;
+  int staged = -1;
+  if (a.xs_all) {
+    stage_x(0, a.xs_cols);
+    staged = 0;
+  }
+  __syncthreads();
+
+  const int my_rt_local = warp / a.ks;            // which of the task's row tiles this warp serves
+  const int my_ks = warp - my_rt_local * a.ks;    // which kernel slab of the chunk
+  const bool warp_active = my_rt_local < a.rtt;
+
+  for (int task = blockIdx.x; task < n_tasks; task += gridDim.x) {
+    const int rg = a.split ? task % n_rg : task;
+    const int ch0 = a.split ? task / n_rg : 0;
+    const int ch1 = a.split ? ch0 + 1 : a.n_chunks;
+    for (int i = threadIdx.x; i < a.rtt * 16 * 8 * NT; i += THREADS) red[i] = 0.f;
+    float d[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) d[n][0] = d[n][1] = d[n][2] = d[n][3] = 0.f;
+    const int rt = rg * a.rtt + my_rt_local;
+    for (int ch = ch0; ch < ch1; ++ch) {
+      if (!a.xs_all && staged != ch) {
+        __syncthreads();
+        stage_x(ch * chunk_cols, chunk_cols);
+        staged = ch;
+      }
+      __syncthreads();
+      const int kslab = ch * a.ks + my_ks;
+      if (!warp_active || rt >= n_rt || kslab >= a.n_kslabs) continue;
+      const int ls = kslab / NT, part = kslab - ls * NT;
+      const int ps0 = part * PS;
+      // B fragments of this kernel slab: x'[batch][sub-vector 64 ls + 4 ps + t], hi and lo
+      uint4 bf[PS][NT];
+      const int col_base = (a.xs_all ? kslab * KSV : (kslab - ch * a.ks) * KSV) * 8;
+#pragma unroll
+      for (int ps = 0; ps < PS; ++ps) {
+        const int col = col_base + (4 * ps + t) * 8;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          int bb, part_lo;
+          if (NT == 1) { bb = g & 3; part_lo = g >> 2; }
+          else { part_lo = n / (NT / 2); bb = (n % (NT / 2)) * 8 + g; }
+          uint4 v = make_uint4(0, 0, 0, 0);
+          if (bb < B) v = *reinterpret_cast<const uint4*>((part_lo ? xl : xh) + (size_t)bb * a.xs_cols + col);
+          bf[ps][n] = v;
+        }
+      }
+      // this kernel slab's fields of rows g and g+8 of the row tile
+      constexpr int NWORDS = (2 * W / NT + 3) / 4 + 1;
+      uint32_t w0[NWORDS], w1[NWORDS];
+      w0[NWORDS - 1] = w1[NWORDS - 1] = 0;
+      const int64_t R0 = (int64_t)rt * 16 + g;
+      const uint8_t* blk0 = L.tcodes + R0 * L.tstride + (int64_t)ls * (8 * W) + t * (2 * W) + ps0 * W / 8;
+      load_sub<W, NT>(blk0, w0);
+      load_sub<W, NT>(blk0 + 8 * L.tstride, w1);
+      // gathers of G pair-steps are issued before their MMAs (hides L2 / shared latency)
+      constexpr int G = (W >= 24 || PS < 8) ? (PS < 4 ? PS : 4) : 8;
+#pragma unroll
+      for (int p0 = 0; p0 < PS; p0 += G) {
+        uint4 c0[G], c1[G], e0[G], e1[G];
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+          const uint32_t f0 = field_of<W>(w0, p0 + j), f1 = field_of<W>(w1, p0 + j);
+          if (CB_SMEM) {
+            c0[j] = cb1s[(f0 & m1) * COPIES + (lane & (COPIES - 1))];
+            c1[j] = cb1s[(f1 & m1) * COPIES + (lane & (COPIES - 1))];
+          } else {
+            c0[j] = __ldg(reinterpret_cast<const uint4*>(L.cb1) + (f0 & m1));
+            c1[j] = __ldg(reinterpret_cast<const uint4*>(L.cb1) + (f1 & m1));
+          }
+          if (L.k2) {
+            if (CB_SMEM) {
+              e0[j] = cb2s[(f0 >> L.bits1) * COPIES + (lane & (COPIES - 1))];
+              e1[j] = cb2s[(f1 >> L.bits1) * COPIES + (lane & (COPIES - 1))];
+            } else {
+              e0[j] = __ldg(reinterpret_cast<const uint4*>(L.cb2) + (f0 >> L.bits1));
+              e1[j] = __ldg(reinterpret_cast<const uint4*>(L.cb2) + (f1 >> L.bits1));
+            }
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+#pragma unroll
+          for (int n = 0; n < NT; ++n) {
+            mma16816(d[n], c0[j].x, c1[j].x, c0[j].y, c1[j].y, bf[p0 + j][n].x, bf[p0 + j][n].y);
+            mma16816(d[n], c0[j].z, c1[j].z, c0[j].w, c1[j].w, bf[p0 + j][n].z, bf[p0 + j][n].w);
+            if (L.k2) {
+              mma16816(d[n], e0[j].x, e1[j].x, e0[j].y, e1[j].y, bf[p0 + j][n].x, bf[p0 + j][n].y);
+              mma16816(d[n], e0[j].z, e1[j].z, e0[j].w, e1[j].w, bf[p0 + j][n].z, bf[p0 + j][n].w);
+            }
+          }
+        }
+      }
+    }
+    // ---- reduce the warps' D fragments: red[rt_local][row][col]
+    if (warp_active) {
+      float* r0 = red + ((size_t)my_rt_local * 16 + g) * (8 * NT);
+      float* r1 = r0 + 8 * (8 * NT);
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        atomicAdd(r0 + n * 8 + 2 * t, d[n][0]);
+        atomicAdd(r0 + n * 8 + 2 * t + 1, d[n][1]);
+        atomicAdd(r1 + n * 8 + 2 * t, d[n][2]);
+        atomicAdd(r1 + n * 8 + 2 * t + 1, d[n][3]);
+      }
+    }
+    __syncthreads();
+    // ---- epilogue: (rtt*16 rows) x batch, sparse correction and outlier block
+    const bool first_chunk = ch0 == 0;
+    const int rows = a.rtt * 16;
+    const int lanes_per_row = THREADS / rows;       // rows * lanes_per_row == THREADS
+    const int rl = threadIdx.x / lanes_per_row, sub = threadIdx.x - rl * lanes_per_row;
+    const int64_t row = (int64_t)rg * rows + rl;
+    const bool row_ok = row < L.n_out;
+    {
+      float spv[BP], ov[BP];
+#pragma unroll
+      for (int b = 0; b < BP; ++b) spv[b] = ov[b] = 0.f;
+      if (first_chunk && row_ok) {
+        if (L.nnz > 0) {
+          const int e_end = L.row_ptr[row + 1];
+          for (int e0 = L.row_ptr[row] + sub; e0 < e_end; e0 += 8 * lanes_per_row) {
+            float dl[8];
+            int jj[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int e = e0 + u * lanes_per_row;
+              dl[u] = e < e_end ? L.delta[e] : 0.f;
+              jj[u] = e < e_end ? (L.col16 ? (int)L.col16[e] : L.col[e]) : 0;
+            }
+#pragma unroll
+            for (int b = 0; b < BP; ++b)
+              if (b < B) {
+                float xv[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) xv[u] = load_as_float(a.x, a.xt, (int64_t)b * L.n_in + jj[u]);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) spv[b] = fmaf(dl[u], xv[u], spv[b]);
+              }
+          }
+        }
+        for (int s = sub; s < L.n_sub_o; s += lanes_per_row) {
+          uint32_t f = read_field(L.codes_o + row * L.stride_o, s, L.bits_o);
+          uint4 u = __ldg(reinterpret_cast<const uint4*>(L.cbo) + f);
+          const __half2* h = reinterpret_cast<const __half2*>(&u);
+          float c[8];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) { float2 f2 = __half22float2(h[k]); c[2 * k] = f2.x; c[2 * k + 1] = f2.y; }
+#pragma unroll
+          for (int b = 0; b < BP; ++b)
+            if (b < B) {
+              float acc = ov[b];
+#pragma unroll
+              for (int k = 0; k < 8; ++k) acc = fmaf(c[k], xo[b * n_o + s * 8 + k], acc);
+              ov[b] = acc;
+            }
+        }
+      }
+      // reduce over the lanes of this row (they are consecutive threads)
+#pragma unroll
+      for (int b = 0; b < BP; ++b) {
+        for (int o = 1; o < lanes_per_row; o <<= 1) {
+          spv[b] += __shfl_xor_sync(0xffffffffu, spv[b], o);
+          ov[b] += __shfl_xor_sync(0xffffffffu, ov[b], o);
+        }
+      }
+      const float rsc = (L.rs && row_ok) ? __half2float(L.rs[row]) : 1.f;
+      const float* rr = red + (size_t)rl * (8 * NT);
+#pragma unroll
+      for (int b = 0; b < BP; ++b) {
+        if (!row_ok || b >= B || (b & (lanes_per_row - 1)) != sub) continue;
+        int nh, nl;
+        if (NT == 1) { nh = b; nl = 4 + b; }
+        else { nh = (b / 8) * 8 + (b % 8); nl = (NT / 2 + b / 8) * 8 + (b % 8); }
+        float body = rr[nh] + rr[nl];
+        float v = fmaf(rsc, body + ov[b], spv[b]);
+        if (a.split) atomicAdd(a.acc + (int64_t)b * L.n_out + row, v);
+        else store_from_float(a.y, a.yt, (int64_t)b * L.n_out + row, v);
+      }
+    }
+    __syncthreads();
+  }
+}
+
+__global__ void k_finalize(const float* __restrict__ acc, int64_t n, void* __restrict__ y, vqlin_dtype yt) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    store_from_float(y, yt, i, acc[i]);
+}
+
+template <int NT, int W, bool CB_SMEM, int COPIES>
+static cudaError_t launch_cfg(const Args& args, size_t smem, int grid, cudaStream_t s) {
+  auto k = k_gemv_tc<NT, W, CB_SMEM, COPIES>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k<<<grid, THREADS, smem, s>>>(args);
+  return cudaGetLastError();
+}
+
+template <int NT, int W>
+static cudaError_t launch_w(const Args& args, bool cb_smem, int copies, size_t smem, int grid, cudaStream_t s) {
+  if (!cb_smem) return launch_cfg<NT, W, false, 1>(args, smem, grid, s);
+  switch (copies) {
+    case 8: return launch_cfg<NT, W, true, 8>(args, smem, grid, s);
+    case 4: return launch_cfg<NT, W, true, 4>(args, smem, grid, s);
+    case 2: return launch_cfg<NT, W, true, 2>(args, smem, grid, s);
+    default: return launch_cfg<NT, W, true, 1>(args, smem, grid, s);
+  }
+}
+
+template <int NT>
+static cudaError_t launch_nt(const Args& args, bool cb_smem, int copies, size_t smem, int grid, cudaStream_t s) {
+  switch (args.L.w) {
+    case 8: return launch_w<NT, 8>(args, cb_smem, copies, smem, grid, s);
+    case 12: return launch_w<NT, 12>(args, cb_smem, copies, smem, grid, s);
+    case 16: return launch_w<NT, 16>(args, cb_smem, copies, smem, grid, s);
+    case 24: return launch_w<NT, 24>(args, cb_smem, copies, smem, grid, s);
+    default: return launch_w<NT, 32>(args, cb_smem, copies, smem, grid, s);
+  }
+}
+
+}  // namespace tcg
+
+bool tc_supported(const Layer& L) {
+  return L.d == 8 && L.tcodes != nullptr && (L.w == 8 || L.w == 12 || L.w == 16 || L.w == 24 || L.w == 32);
+}
+
+size_t gemv_workspace_bytes(const Layer& L, int batch) {
+  return ((size_t)batch * L.n_out * 4 + 255) & ~size_t(255);
+}
+
+// Plan and launch.  acc_ws: caller workspace for split accumulation (may be null).
+cudaError_t launch_gemv_tc(const Layer& L, const void* x, vqlin_dtype xt, int batch, void* y, vqlin_dtype yt,
+                           void* ws, size_t ws_bytes, cudaStream_t s, bool* handled) {
+  using namespace tcg;
+  *handled = false;
+  if (!tc_supported(L) || batch < 1 || batch > 16) return cudaSuccess;
+  const int NT = batch <= 4 ? 1 : (batch <= 8 ? 2 : 4);
+  const int KSV = 64 / NT;
+  const int BP = 4 * NT;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const size_t smem_max = 227 * 1024;
+  // codebooks: as many interleaved copies (<= 8) as fit next to x'
+  const size_t cb_entries = (size_t)L.k1 + L.k2;
+  Args a;
+  a.L = L; a.x = x; a.xt = xt; a.batch = batch; a.y = y; a.yt = yt; a.acc = nullptr;
+  a.n_kslabs = (L.n_sub + KSV - 1) / KSV;
+  a.ks = a.n_kslabs < WARPS ? a.n_kslabs : WARPS;
+  // round ks down to a divisor of WARPS so that rtt * ks == WARPS when several row tiles share a CTA
+  while (WARPS % a.ks) --a.ks;
+  a.rtt = WARPS / a.ks;
+  a.n_chunks = (a.n_kslabs + a.ks - 1) / a.ks;
+  const size_t red_bytes = (size_t)a.rtt * 16 * 8 * NT * 4;
+  const size_t xo_bytes = (size_t)BP * L.n_sub_o * 8 * 4;
+  const int all_cols = a.n_kslabs * KSV * 8;
+  const int chunk_cols = a.ks * KSV * 8;
+  const size_t x_all = (size_t)batch * all_cols * 4, x_chunk = (size_t)batch * chunk_cols * 4;
+  // choose codebook placement and x' staging
+  int copies = 0;
+  bool cb_smem = false;
+  for (int c = 8; c >= 1; c >>= 1) {
+    size_t need = cb_entries * 16 * c + red_bytes + xo_bytes + x_chunk + 256;
+    if (need <= smem_max && cb_entries * 16 * c <= 160 * 1024) { copies = c; cb_smem = true; break; }
+  }
+  const size_t cb_bytes = cb_smem ? cb_entries * 16 * copies : 0;
+  a.xs_all = (cb_bytes + red_bytes + xo_bytes + x_all + 256 <= smem_max) ? 1 : 0;
+  a.xs_cols = a.xs_all ? all_cols : chunk_cols;
+  const size_t smem = cb_bytes + (size_t)batch * a.xs_cols * 4 + red_bytes + xo_bytes + 64;
+  if (smem > smem_max) return cudaSuccess;   // does not fit: caller uses the generic kernel
+  const int n_rt = (L.n_out + 15) / 16;
+  const int n_rg = (n_rt + a.rtt - 1) / a.rtt;
+  // split by chunk when there is more than one chunk and a fp32 accumulator is available
+  a.split = 0;
+  if (a.n_chunks > 1) {
+    if (yt == VQLIN_F32) { a.split = 1; a.acc = reinterpret_cast<float*>(y); }
+    else if (ws && ws_bytes >= gemv_workspace_bytes(L, batch)) { a.split = 1; a.acc = reinterpret_cast<float*>(ws); }
+    // otherwise every task loops over the chunks itself (no scratch needed)
+  }
+  const int n_tasks = a.split ? n_rg * a.n_chunks : n_rg;
+  const int per_sm = (int)(smem_max / (smem + 1024)) < 1 ? 1 : (int)(smem_max / (smem + 1024));
+  int grid = sms * (per_sm > 2 ? 2 : per_sm);
+  if (grid > n_tasks) grid = n_tasks;
+  cudaError_t e;
+  if (a.split) {
+    e = cudaMemsetAsync(a.acc, 0, (size_t)batch * L.n_out * 4, s);
+    if (e != cudaSuccess) return e;
+  }
+  if (NT == 1) e = launch_nt<1>(a, cb_smem, copies, smem, grid, s);
+  else if (NT == 2) e = launch_nt<2>(a, cb_smem, copies, smem, grid, s);
+  else e = launch_nt<4>(a, cb_smem, copies, smem, grid, s);
+  if (e != cudaSuccess) return e;
+  if (a.split && yt != VQLIN_F32) {
+    int64_t n = (int64_t)batch * L.n_out;
+    k_finalize<<<(int)((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024), 256, 0, s>>>(a.acc, n, y, yt);
+    e = cudaGetLastError();
+  }
+  *handled = (e == cudaSuccess);
+  return e;
+}
+
+}  // namespace vqlin

@@ -34,6 +34,12 @@ struct Layer {
   const uint16_t* val;                  // [nnz] fp16 bits (exact replacement values)
   const float* delta;                   // [nnz] v - body, for the fused products
   const uint16_t* col16;                // [nnz] column ids as u16 when n_in <= 65536, else null
+  // Tensor-core decode layout (d = 8, w in {8,12,16,24,32}; null otherwise): rows padded
+  // to a multiple of 16; per row and per slab of 64 sub-vectors, for t = 0..3 the 16
+  // fields of sub-vectors 64*slab + 4*ps + t (ps = 0..15), packed LSB-first.
+  const uint8_t* tcodes;
+  int32_t n_ls;                         // layout slabs per row
+  int64_t tstride;                      // bytes per row = n_ls * 8 * w
 };
 
 // Last-error plumbing (thread-local detail string).
@@ -44,7 +50,13 @@ vqlin_status cuda_status(cudaError_t e, const char* what);
 cudaError_t launch_unpack(const Layer& L, int which, uint32_t* out, cudaStream_t s);
 cudaError_t launch_dequant(const Layer& L, __half* W, int64_t ldw, cudaStream_t s);
 cudaError_t launch_gemv(const Layer& L, const void* x, vqlin_dtype xt, int batch, void* y, vqlin_dtype yt,
-                        cudaStream_t s);
+                        void* ws, size_t ws_bytes, cudaStream_t s);
+bool tc_supported(const Layer& L);
+size_t gemv_workspace_bytes(const Layer& L, int batch);
+cudaError_t launch_gemv_tc(const Layer& L, const void* x, vqlin_dtype xt, int batch, void* y, vqlin_dtype yt,
+                           void* ws, size_t ws_bytes, cudaStream_t s, bool* handled);
+cudaError_t launch_gemv_generic(const Layer& L, const void* x, vqlin_dtype xt, int batch, void* y, vqlin_dtype yt,
+                                cudaStream_t s);
 cudaError_t launch_convert_to_f16(const void* X, vqlin_dtype xt, int64_t n, __half* out, cudaStream_t s);
 int read_and_clear_device_error();
 cudaError_t launch_gemm_f16(const __half* A, const __half* W, int64_t M, int N, int K, void* Y, vqlin_dtype yt,

@@ -74,6 +74,8 @@ vqlin_destroy = _sig("vqlin_destroy", _S, [_H])
 vqlin_get_info = _sig("vqlin_get_info", _S, [_H, C.POINTER(vqlin_info)])
 vqlin_dequant = _sig("vqlin_dequant", _S, [_H, _P, C.c_int64, _P])
 vqlin_gemv = _sig("vqlin_gemv", _S, [_H, _P, C.c_int, C.c_int32, _P, C.c_int, _P])
+vqlin_gemv_ws = _sig("vqlin_gemv_ws", _S, [_H, _P, C.c_int, C.c_int32, _P, C.c_int, _P, C.c_size_t, _P])
+vqlin_gemv_workspace_size = _sig("vqlin_gemv_workspace_size", C.c_size_t, [_H, C.c_int32])
 vqlin_gemm = _sig("vqlin_gemm", _S, [_H, _P, C.c_int, C.c_int64, _P, C.c_int, _P, C.c_size_t, _P])
 vqlin_gemm_workspace_size = _sig("vqlin_gemm_workspace_size", C.c_size_t, [_H, C.c_int64])
 vqlin_unpack_indices = _sig("vqlin_unpack_indices", _S, [_H, C.c_int32, _P, _P])
@@ -84,7 +86,7 @@ vqlin_device_error = _sig("vqlin_device_error", _S, [C.POINTER(C.c_int32)])
 
 EXPORTS = ["vqlin_create", "vqlin_destroy", "vqlin_get_info", "vqlin_dequant", "vqlin_gemv", "vqlin_gemm",
            "vqlin_gemm_workspace_size", "vqlin_unpack_indices", "vqlin_status_string", "vqlin_last_error",
-           "vqlin_abi_version", "vqlin_device_error"]
+           "vqlin_abi_version", "vqlin_device_error", "vqlin_gemv_ws", "vqlin_gemv_workspace_size"]
 
 
 def device_error() -> int:
@@ -215,6 +217,19 @@ class VQLinear:
             out = torch.empty((x2.shape[0], self.n_out), dtype=out_dtype or torch.float32, device=x.device)
         check(vqlin_gemv(self._h, x2.data_ptr(), dtype_code(x2.dtype), x2.shape[0], out.data_ptr(),
                          dtype_code(out.dtype), _stream(stream)), "vqlin_gemv")
+        return out
+
+    def gemv_ws(self, x, workspace=None, out=None, out_dtype=None, stream=None):
+        import torch
+        x2 = x if x.dim() == 2 else x.view(1, -1)
+        assert x2.is_contiguous() and x2.shape[1] == self.n_in
+        B = x2.shape[0]
+        if out is None:
+            out = torch.empty((B, self.n_out), dtype=out_dtype or torch.float32, device=x.device)
+        if workspace is None:
+            workspace = torch.empty(int(vqlin_gemv_workspace_size(self._h, B)), dtype=torch.uint8, device=x.device)
+        check(vqlin_gemv_ws(self._h, x2.data_ptr(), dtype_code(x2.dtype), B, out.data_ptr(), dtype_code(out.dtype),
+                            workspace.data_ptr(), workspace.numel(), _stream(stream)), "vqlin_gemv_ws")
         return out
 
     def workspace_size(self, m: int) -> int:

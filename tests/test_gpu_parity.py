@@ -323,3 +323,41 @@ def test_device_pointers_create(vq):
                              for k, v in L.__dict__.items()})
     W = vq.VQLinear(dev).dequant().cpu().numpy().view(np.uint16)
     assert (W == oracle.dequant_exact(L)).all()
+
+
+# ------------------------------------------------------------------ gemv with a caller workspace (split columns)
+@pytest.mark.parametrize("name,batch,ydt", [("downproj", 1, "f16"), ("downproj", 16, "bf16"), ("smollm:6", 8, "f16"),
+                                            ("qproj", 4, "f16"), ("smollm:0", 1, "f32")])
+def test_gemv_ws_full(vq, name, batch, ydt):
+    import torch
+    L = full_layer(name)
+    if name.startswith("smollm"):
+        xb = G.workload("smollm")[1][int(name.split(":")[1])][:batch]
+        xdt = "bf16"
+    else:
+        xb = G.workload(name)[1][:batch]
+        xdt = "f16"
+    m = vq.VQLinear(L)
+    x = G.torch_x(xb, xdt)
+    ws = torch.full((m_ws := int(vq.vqlin_gemv_workspace_size(m.handle, batch)),), 0x7F, dtype=torch.uint8, device="cuda")
+    y = m.gemv_ws(x, workspace=ws, out_dtype=G.torch_dtype(ydt))
+    y2 = m.gemv(x, out_dtype=G.torch_dtype(ydt))
+    torch.cuda.synchronize()
+    ref = oracle.gemv_f64(L, synth.bits_to_f64(xb, xdt))
+    G.assert_close(G.to_f64(y), ref, ydt, "gemv_ws %s B=%d" % (name, batch))
+    G.assert_close(G.to_f64(y2), ref, ydt, "gemv %s B=%d" % (name, batch))
+    assert m_ws >= batch * L.n_out * 4
+
+
+def test_gemv_ws_errors(vq):
+    import torch
+    L = SMALL[1]
+    m = vq.VQLinear(L)
+    x = torch.zeros((2, L.n_in), dtype=torch.float16, device="cuda")
+    y = torch.zeros((2, L.n_out), dtype=torch.float16, device="cuda")
+    need = int(vq.vqlin_gemv_workspace_size(m.handle, 2))
+    ws = torch.zeros(need + 256, dtype=torch.uint8, device="cuda")
+    assert vq.vqlin_gemv_ws(m.handle, x.data_ptr(), vq.VQLIN_F16, 2, y.data_ptr(), vq.VQLIN_F16, ws.data_ptr(), need - 1, None) == vq.VQLIN_ERR_WORKSPACE
+    assert vq.vqlin_gemv_ws(m.handle, x.data_ptr(), vq.VQLIN_F16, 2, y.data_ptr(), vq.VQLIN_F16, ws.data_ptr() + 16, need, None) == vq.VQLIN_ERR_WORKSPACE
+    assert vq.vqlin_gemv_ws(m.handle, x.data_ptr(), vq.VQLIN_F16, 2, y.data_ptr(), vq.VQLIN_F16, ws.data_ptr(), need, None) == vq.VQLIN_OK
+    torch.cuda.synchronize()
