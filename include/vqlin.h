@@ -205,6 +205,24 @@ vqlin_status vqlin_gemv_ws(const vqlin_handle* h, const void* x, vqlin_dtype xt,
 size_t vqlin_gemv_workspace_size(const vqlin_handle* h, int32_t batch);
 
 /*
+ * The decode GEMV for callers that cannot allocate device memory at call time
+ * (a serving loop whose pool already owns the GPU's memory, a path where
+ * cudaMalloc's implicit device synchronisation is not allowed, a plug-in that
+ * may only touch the buffers it is handed).  It computes what vqlin_gemv_ws
+ * computes, but its column-split accumulator is a scratch array built into the
+ * library (1 MiB of fp32 per device, held until the process exits) instead of
+ * a caller buffer, and it allocates nothing.  Limit: batch * n_out <= 262144,
+ * else VQLIN_ERR_UNSUPPORTED.  The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress) and caches it: make that first call
+ * outside stream capture.  All calls share the array: calls whose kernels
+ * overlap on the GPU race on it, so the caller must serialise them.  The array
+ * is cleared on the call's stream before each use.  (No counterpart on the
+ * pages: this is an interface convenience.)
+ */
+vqlin_status vqlin_gemv_noalloc(const vqlin_handle* h, const void* x, vqlin_dtype xt, int32_t batch,
+                                void* y, vqlin_dtype yt, void* stream);
+
+/*
  * Prefill: Y[m*n_out + i] = sum_j W[i,j] * X[m*n_in + j] for 0 <= m < M.
  * X: device [M][n_in] of xt (F16 or BF16; BF16 is converted to fp16, exact for
  * 2^-14 <= |x| <= 65504), Y: device [M][n_out] of yt.  The weight enters the

@@ -76,6 +76,7 @@ vqlin_dequant = _sig("vqlin_dequant", _S, [_H, _P, C.c_int64, _P])
 vqlin_gemv = _sig("vqlin_gemv", _S, [_H, _P, C.c_int, C.c_int32, _P, C.c_int, _P])
 vqlin_gemv_ws = _sig("vqlin_gemv_ws", _S, [_H, _P, C.c_int, C.c_int32, _P, C.c_int, _P, C.c_size_t, _P])
 vqlin_gemv_workspace_size = _sig("vqlin_gemv_workspace_size", C.c_size_t, [_H, C.c_int32])
+vqlin_gemv_noalloc = _sig("vqlin_gemv_noalloc", _S, [_H, _P, C.c_int, C.c_int32, _P, C.c_int, _P])
 vqlin_gemm = _sig("vqlin_gemm", _S, [_H, _P, C.c_int, C.c_int64, _P, C.c_int, _P, C.c_size_t, _P])
 vqlin_gemm_workspace_size = _sig("vqlin_gemm_workspace_size", C.c_size_t, [_H, C.c_int64])
 vqlin_unpack_indices = _sig("vqlin_unpack_indices", _S, [_H, C.c_int32, _P, _P])
@@ -86,7 +87,7 @@ vqlin_device_error = _sig("vqlin_device_error", _S, [C.POINTER(C.c_int32)])
 
 EXPORTS = ["vqlin_create", "vqlin_destroy", "vqlin_get_info", "vqlin_dequant", "vqlin_gemv", "vqlin_gemm",
            "vqlin_gemm_workspace_size", "vqlin_unpack_indices", "vqlin_status_string", "vqlin_last_error",
-           "vqlin_abi_version", "vqlin_device_error", "vqlin_gemv_ws", "vqlin_gemv_workspace_size"]
+           "vqlin_abi_version", "vqlin_device_error", "vqlin_gemv_ws", "vqlin_gemv_workspace_size", "vqlin_gemv_noalloc"]
 
 
 def device_error() -> int:
