@@ -258,6 +258,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
       load_sub<W, NT>(blk0 + 8 * L.tstride, w1);
       // gathers of G pair-steps are issued before their MMAs (hides L2 / shared latency)
       constexpr int G = (W >= 24 || PS < 8) ? (PS < 4 ? PS : 4) : 8;
+      static_assert(PS % G == 0 && G <= PS, "pair-step batches must tile the kernel slab");
 #pragma unroll
       for (int p0 = 0; p0 < PS; p0 += G) {
         uint4 c0[G], c1[G], e0[G], e1[G];
@@ -385,6 +386,280 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Warp-task variant.  Every (16-row tile, kernel slab) is an independent warp
+// task that adds r * (its partial dot products) to a zeroed fp32 accumulator
+// with atomics; every group of 8 rows has a task for the fused sparse term and
+// the outlier block.  The sparse tasks come first in the task order so their
+// dependent loads overlap the MMA tasks.  Shared memory holds the codebooks and
+// x' for every column, written once; after that no block-wide barrier is needed,
+// so warps overlap each other's memory latency freely.  B fragments are read
+// from shared memory per pair-step, which keeps registers low enough for two
+// blocks per SM.
+template <int NT, int W, bool CB_SMEM, int COPIES>
+__global__ void __launch_bounds__(THREADS, 2) k_gemv_wt(Args a) {
+  constexpr int PS = 16 / NT;
+  constexpr int KSV = 4 * PS;
+  constexpr int BP = 4 * NT;
+  const Layer& L = a.L;
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint4* cb1s = reinterpret_cast<uint4*>(smem);
+  uint4* cb2s = cb1s + (CB_SMEM ? (size_t)L.k1 * COPIES : 0);
+  __half* xh = reinterpret_cast<__half*>(cb2s + (CB_SMEM ? (size_t)L.k2 * COPIES : 0));   // [batch][xs_cols]
+  __half* xl = xh + (size_t)a.batch * a.xs_cols;
+  float* xo = reinterpret_cast<float*>(xl + (size_t)a.batch * a.xs_cols);               // [BP][n_sub_o*8]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int B = a.batch;
+  const uint32_t m1 = (1u << L.bits1) - 1u;
+
+  if (CB_SMEM) {
+    const uint4* c1 = reinterpret_cast<const uint4*>(L.cb1);
+    for (int i = threadIdx.x; i < L.k1 * COPIES; i += THREADS) cb1s[i] = __ldg(c1 + i / COPIES);
+    if (L.k2) {
+      const uint4* c2 = reinterpret_cast<const uint4*>(L.cb2);
+      for (int i = threadIdx.x; i < L.k2 * COPIES; i += THREADS) cb2s[i] = __ldg(c2 + i / COPIES);
+    }
+  }
+  const int n_o = L.n_sub_o * 8;
+  for (int i = threadIdx.x; i < BP * n_o; i += THREADS) {
+    int b = i / n_o, p = i - b * n_o;
+    float v = 0.f;
+    if (b < B && p < L.n_ocols) {
+      int j = L.colmap[L.n_main + p];
+      v = load_as_float(a.x, a.xt, (int64_t)b * L.n_in + j);
+      if (L.cs) v *= __half2float(L.cs[j]);
+    }
+    xo[i] = v;
+  }
+  // x' hi/lo for every main column, eight columns per thread, loads first
+  {
+    const int groups = a.xs_cols / 8;
+    for (int i = threadIdx.x; i < B * groups; i += THREADS) {
+      const int b = i / groups, q = (i - b * groups) * 8;
+      float v[8];
+      if (!L.colmap && a.xt != VQLIN_F32 && q + 8 <= L.n_main && (L.n_in & 7) == 0) {
+        uint4 u = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const unsigned short*>(a.x) +
+                                                        (int64_t)b * L.n_in + q));
+        const unsigned short* hs = reinterpret_cast<const unsigned short*>(&u);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          v[k] = a.xt == VQLIN_F16 ? __half2float(__ushort_as_half(hs[k])) : __bfloat162float(__ushort_as_bfloat16(hs[k]));
+        if (L.cs) {
+          uint4 cu = __ldg(reinterpret_cast<const uint4*>(L.cs + q));
+          const __half* cv = reinterpret_cast<const __half*>(&cu);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) v[k] *= __half2float(cv[k]);
+        }
+      } else {
+        int jj[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) jj[k] = q + k < L.n_main ? (L.colmap ? L.colmap[q + k] : q + k) : -1;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = jj[k] >= 0 ? load_as_float(a.x, a.xt, (int64_t)b * L.n_in + jj[k]) : 0.f;
+        if (L.cs) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) v[k] *= jj[k] >= 0 ? __half2float(L.cs[jj[k]]) : 0.f;
+        }
+      }
+      uint32_t ph[4], pl[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        __half h0 = __float2half_rn(v[2 * k]), h1 = __float2half_rn(v[2 * k + 1]);
+        __half l0 = __float2half_rn(v[2 * k] - __half2float(h0)), l1 = __float2half_rn(v[2 * k + 1] - __half2float(h1));
+        ph[k] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16);
+        pl[k] = (uint32_t)__half_as_ushort(l0) | ((uint32_t)__half_as_ushort(l1) << 16);
+      }
+      *reinterpret_cast<uint4*>(xh + (size_t)b * a.xs_cols + q) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+      *reinterpret_cast<uint4*>(xl + (size_t)b * a.xs_cols + q) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+    }
+  }
+  __syncthreads();
+
+  const int n_rt = (L.n_out + 15) / 16;
+  const bool has_side = L.nnz > 0 || L.n_ocols > 0;
+  const int n_side = has_side ? (L.n_out + 7) / 8 : 0;      // sparse / outlier tasks of 8 rows
+  const int n_main = n_rt * a.n_kslabs;
+  const int total = n_side + n_main;
+  for (int task = blockIdx.x * WARPS + warp; task < total; task += gridDim.x * WARPS) {
+    if (task < n_side) {
+      // ---- fused sparse correction and outlier block for rows 8*task .. +8 (4 lanes per row)
+      const int64_t row = (int64_t)task * 8 + (lane >> 2);
+      const int sub = lane & 3;
+      const bool ok = row < L.n_out;
+      float spv[BP], ov[BP];
+#pragma unroll
+      for (int b = 0; b < BP; ++b) spv[b] = ov[b] = 0.f;
+      if (ok && L.nnz > 0) {
+        const int e_end = L.row_ptr[row + 1];
+        for (int e0 = L.row_ptr[row] + sub; e0 < e_end; e0 += 32) {
+          float dl[8];
+          int jj[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int e = e0 + 4 * u;
+            dl[u] = e < e_end ? L.delta[e] : 0.f;
+            jj[u] = e < e_end ? (L.col16 ? (int)L.col16[e] : L.col[e]) : 0;
+          }
+#pragma unroll
+          for (int b = 0; b < BP; ++b)
+            if (b < B) {
+              float xv[8];
+#pragma unroll
+              for (int u = 0; u < 8; ++u) xv[u] = load_as_float(a.x, a.xt, (int64_t)b * L.n_in + jj[u]);
+#pragma unroll
+              for (int u = 0; u < 8; ++u) spv[b] = fmaf(dl[u], xv[u], spv[b]);
+            }
+        }
+      }
+      if (ok) {
+        for (int so = sub; so < L.n_sub_o; so += 4) {
+          uint32_t f = read_field(L.codes_o + row * L.stride_o, so, L.bits_o);
+          uint4 u = __ldg(reinterpret_cast<const uint4*>(L.cbo) + f);
+          const __half2* h = reinterpret_cast<const __half2*>(&u);
+          float c[8];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) { float2 f2 = __half22float2(h[k]); c[2 * k] = f2.x; c[2 * k + 1] = f2.y; }
+#pragma unroll
+          for (int b = 0; b < BP; ++b)
+            if (b < B) {
+              float acc = ov[b];
+#pragma unroll
+              for (int k = 0; k < 8; ++k) acc = fmaf(c[k], xo[b * n_o + so * 8 + k], acc);
+              ov[b] = acc;
+            }
+        }
+      }
+      const float rsc = (ok && L.rs) ? __half2float(L.rs[row]) : 1.f;
+#pragma unroll
+      for (int b = 0; b < BP; ++b) {
+        float v = fmaf(rsc, ov[b], spv[b]);
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        if (ok && b < B && sub == (b & 3) && v != 0.f) atomicAdd(a.acc + (int64_t)b * L.n_out + row, v);
+      }
+      continue;
+    }
+    // ---- MMA task: row tile rt, kernel slab ks
+    const int mt = task - n_side;
+    const int rt = mt / a.n_kslabs, kslab = mt - rt * a.n_kslabs;
+    const int ls = kslab / NT, part = kslab - ls * NT;
+    const int64_t R0 = (int64_t)rt * 16 + g;
+    constexpr int NWORDS = (2 * W / NT + 3) / 4 + 1;
+    uint32_t w0[NWORDS], w1[NWORDS];
+    w0[NWORDS - 1] = w1[NWORDS - 1] = 0;
+    const uint8_t* blk0 = L.tcodes + R0 * L.tstride + (int64_t)ls * (8 * W) + t * (2 * W) + part * PS * W / 8;
+    load_sub<W, NT>(blk0, w0);
+    load_sub<W, NT>(blk0 + 8 * L.tstride, w1);
+    const float r0 = (L.rs && R0 < L.n_out) ? __half2float(L.rs[R0]) : 1.f;
+    const float r1 = (L.rs && R0 + 8 < L.n_out) ? __half2float(L.rs[R0 + 8]) : 1.f;
+    float d[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) d[n][0] = d[n][1] = d[n][2] = d[n][3] = 0.f;
+    const int col_base = kslab * KSV * 8;
+    // gathers per batch: never more than the slab's pair-steps (PS is 4 when NT = 4)
+    constexpr int G = ((W >= 24) ? 4 : 8) < PS ? ((W >= 24) ? 4 : 8) : PS;
+    static_assert(PS % G == 0, "pair-step batches must tile the kernel slab");
+#pragma unroll
+    for (int p0 = 0; p0 < PS; p0 += G) {
+      uint4 c0[G], c1[G], e0[G], e1[G];
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        const uint32_t f0 = field_of<W>(w0, p0 + j), f1 = field_of<W>(w1, p0 + j);
+        if (CB_SMEM) {
+          c0[j] = cb1s[(f0 & m1) * COPIES + (lane & (COPIES - 1))];
+          c1[j] = cb1s[(f1 & m1) * COPIES + (lane & (COPIES - 1))];
+        } else {
+          c0[j] = __ldg(reinterpret_cast<const uint4*>(L.cb1) + (f0 & m1));
+          c1[j] = __ldg(reinterpret_cast<const uint4*>(L.cb1) + (f1 & m1));
+        }
+        if (L.k2) {
+          if (CB_SMEM) {
+            e0[j] = cb2s[(f0 >> L.bits1) * COPIES + (lane & (COPIES - 1))];
+            e1[j] = cb2s[(f1 >> L.bits1) * COPIES + (lane & (COPIES - 1))];
+          } else {
+            e0[j] = __ldg(reinterpret_cast<const uint4*>(L.cb2) + (f0 >> L.bits1));
+            e1[j] = __ldg(reinterpret_cast<const uint4*>(L.cb2) + (f1 >> L.bits1));
+          }
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        const int col = col_base + (4 * (p0 + j) + t) * 8;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          int bb, part_lo;
+          if (NT == 1) { bb = g & 3; part_lo = g >> 2; }
+          else { part_lo = n / (NT / 2); bb = (n % (NT / 2)) * 8 + g; }
+          uint4 bv = make_uint4(0, 0, 0, 0);
+          if (bb < B) bv = *reinterpret_cast<const uint4*>((part_lo ? xl : xh) + (size_t)bb * a.xs_cols + col);
+          mma16816(d[n], c0[j].x, c1[j].x, c0[j].y, c1[j].y, bv.x, bv.y);
+          mma16816(d[n], c0[j].z, c1[j].z, c0[j].w, c1[j].w, bv.z, bv.w);
+          if (L.k2) {
+            mma16816(d[n], e0[j].x, e1[j].x, e0[j].y, e1[j].y, bv.x, bv.y);
+            mma16816(d[n], e0[j].z, e1[j].z, e0[j].w, e1[j].w, bv.z, bv.w);
+          }
+        }
+      }
+    }
+    // hi + lo, times the row scale, into the accumulator
+    if (NT == 1) {
+      // columns 0-3 hold hi of batches 0-3, columns 4-7 lo: lanes t and t^2 pair up
+#pragma unroll
+      for (int k = 0; k < 4; ++k) d[0][k] += __shfl_xor_sync(0xffffffffu, d[0][k], 2);
+      if (t < 2) {
+        const int b0 = 2 * t, b1 = 2 * t + 1;
+        if (b0 < B && R0 < L.n_out) atomicAdd(a.acc + (int64_t)b0 * L.n_out + R0, r0 * d[0][0]);
+        if (b1 < B && R0 < L.n_out) atomicAdd(a.acc + (int64_t)b1 * L.n_out + R0, r0 * d[0][1]);
+        if (b0 < B && R0 + 8 < L.n_out) atomicAdd(a.acc + (int64_t)b0 * L.n_out + R0 + 8, r1 * d[0][2]);
+        if (b1 < B && R0 + 8 < L.n_out) atomicAdd(a.acc + (int64_t)b1 * L.n_out + R0 + 8, r1 * d[0][3]);
+      }
+    } else {
+#pragma unroll
+      for (int h = 0; h < NT / 2; ++h) {
+        const int b0 = h * 8 + 2 * t, b1 = b0 + 1;
+        const float v00 = d[h][0] + d[NT / 2 + h][0], v01 = d[h][1] + d[NT / 2 + h][1];
+        const float v10 = d[h][2] + d[NT / 2 + h][2], v11 = d[h][3] + d[NT / 2 + h][3];
+        if (b0 < B && R0 < L.n_out) atomicAdd(a.acc + (int64_t)b0 * L.n_out + R0, r0 * v00);
+        if (b1 < B && R0 < L.n_out) atomicAdd(a.acc + (int64_t)b1 * L.n_out + R0, r0 * v01);
+        if (b0 < B && R0 + 8 < L.n_out) atomicAdd(a.acc + (int64_t)b0 * L.n_out + R0 + 8, r1 * v10);
+        if (b1 < B && R0 + 8 < L.n_out) atomicAdd(a.acc + (int64_t)b1 * L.n_out + R0 + 8, r1 * v11);
+      }
+    }
+  }
+}
+
+template <int NT, int W, bool CB_SMEM, int COPIES>
+static cudaError_t launch_wt_cfg(const Args& args, size_t smem, int grid, cudaStream_t s) {
+  auto k = k_gemv_wt<NT, W, CB_SMEM, COPIES>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k<<<grid, THREADS, smem, s>>>(args);
+  return cudaGetLastError();
+}
+
+template <int NT, int W>
+static cudaError_t launch_wt_w(const Args& args, bool cb_smem, int copies, size_t smem, int grid, cudaStream_t s) {
+  if (!cb_smem) return launch_wt_cfg<NT, W, false, 1>(args, smem, grid, s);
+  switch (copies) {
+    case 8: return launch_wt_cfg<NT, W, true, 8>(args, smem, grid, s);
+    case 4: return launch_wt_cfg<NT, W, true, 4>(args, smem, grid, s);
+    case 2: return launch_wt_cfg<NT, W, true, 2>(args, smem, grid, s);
+    default: return launch_wt_cfg<NT, W, true, 1>(args, smem, grid, s);
+  }
+}
+
+template <int NT>
+static cudaError_t launch_wt_nt(const Args& args, bool cb_smem, int copies, size_t smem, int grid, cudaStream_t s) {
+  switch (args.L.w) {
+    case 8: return launch_wt_w<NT, 8>(args, cb_smem, copies, smem, grid, s);
+    case 12: return launch_wt_w<NT, 12>(args, cb_smem, copies, smem, grid, s);
+    case 16: return launch_wt_w<NT, 16>(args, cb_smem, copies, smem, grid, s);
+    case 24: return launch_wt_w<NT, 24>(args, cb_smem, copies, smem, grid, s);
+    default: return launch_wt_w<NT, 32>(args, cb_smem, copies, smem, grid, s);
+  }
+}
+
 __global__ void k_finalize(const float* __restrict__ acc, int64_t n, void* __restrict__ y, vqlin_dtype yt) {
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
     store_from_float(y, yt, i, acc[i]);
@@ -473,7 +748,47 @@ cudaError_t launch_gemv_tc(const Layer& L, const void* x, vqlin_dtype xt, int ba
   if (smem > smem_max) return cudaSuccess;   // does not fit: caller uses the generic kernel
   const int n_rt = (L.n_out + 15) / 16;
   const int n_rg = (n_rt + a.rtt - 1) / a.rtt;
-  // split by chunk when there is more than one chunk and a fp32 accumulator is available
+  // ---- warp-task kernel: needs an fp32 accumulator (y itself, or the caller's workspace)
+  //      and x' for every column next to the codebooks
+  {
+    float* acc = nullptr;
+    if (yt == VQLIN_F32) acc = reinterpret_cast<float*>(y);
+    else if (ws && ws_bytes >= gemv_workspace_bytes(L, batch)) acc = reinterpret_cast<float*>(ws);
+    int wcopies = 0;
+    bool wcb = false;
+    for (int c = 8; c >= 1; c >>= 1) {
+      if (cb_entries * 16 * c <= 160 * 1024 && cb_entries * 16 * c + x_all + xo_bytes + 256 <= smem_max) {
+        wcopies = c; wcb = true; break;
+      }
+    }
+    const size_t wsmem = (wcb ? cb_entries * 16 * wcopies : 0) + x_all + xo_bytes + 64;
+    if (acc && wsmem <= smem_max) {
+      Args w = a;
+      w.acc = acc;
+      w.xs_all = 1;
+      w.xs_cols = all_cols;
+      const int n_side = (L.nnz > 0 || L.n_ocols > 0) ? (L.n_out + 7) / 8 : 0;
+      const int total = n_side + n_rt * a.n_kslabs;
+      const int per_sm = (int)(smem_max / (wsmem + 1024)) >= 2 ? 2 : 1;
+      int grid = sms * per_sm;
+      if (grid > (total + WARPS - 1) / WARPS) grid = (total + WARPS - 1) / WARPS;
+      cudaError_t e = cudaMemsetAsync(acc, 0, (size_t)batch * L.n_out * 4, s);
+      if (e != cudaSuccess) return e;
+      if (NT == 1) e = launch_wt_nt<1>(w, wcb, wcopies, wsmem, grid, s);
+      else if (NT == 2) e = launch_wt_nt<2>(w, wcb, wcopies, wsmem, grid, s);
+      else e = launch_wt_nt<4>(w, wcb, wcopies, wsmem, grid, s);
+      if (e != cudaSuccess) return e;
+      if (yt != VQLIN_F32) {
+        int64_t n = (int64_t)batch * L.n_out;
+        k_finalize<<<(int)((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024), 256, 0, s>>>(acc, n, y, yt);
+        e = cudaGetLastError();
+      }
+      *handled = (e == cudaSuccess);
+      return e;
+    }
+  }
+  // ---- block-task kernel (no scratch needed); split by chunk when there is more than one chunk
+  //      and an fp32 accumulator is available
   a.split = 0;
   if (a.n_chunks > 1) {
     if (yt == VQLIN_F32) { a.split = 1; a.acc = reinterpret_cast<float*>(y); }
