@@ -116,8 +116,9 @@ vqlin_status vqlin_device_error(int32_t* code) {
   vqlin_status st = cuda_status(cudaDeviceSynchronize(), "device synchronize");
   if (st) return st;
   int v = read_and_clear_device_error();
-  if (v < 0) { set_error("cannot read the device error word"); return VQLIN_ERR_CUDA; }
-  *code = v;
+  int w = read_and_clear_cs_error();
+  if (v < 0 || w < 0) { set_error("cannot read the device error words"); return VQLIN_ERR_CUDA; }
+  *code = v ? v : w;
   return VQLIN_OK;
 }
 int32_t vqlin_abi_version(void) { return VQLIN_ABI_VERSION; }
@@ -326,6 +327,57 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
     }
   }
 
+  // codebook-stationary layout for large single-stage codebooks (see vqlin_internal.cuh)
+  std::vector<uint64_t> cs_words;
+  std::vector<int64_t> cs_start;
+  std::vector<uint16_t> cs_counts, cs_wpos;
+  int32_t cs_P = 0, cs_H = 0, cs_E = 0, cs_rpp = 0, cs_lbits = 0, cs_ebits = 0, cs_epw = 0;
+  if (d == 8 && D->k2 == 0 && D->k1 > 10240 && n_sub > 0) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    auto bitlen = [](int64_t v) { int b = 0; while ((1ll << b) <= v) ++b; return b < 1 ? 1 : b; };
+    int H = D->n_out >= 2048 ? 2 : 1;
+    int P = (int)std::max<int64_t>(ceil_div(D->k1, 1024), std::max(1, sms / H));
+    P = std::min(P, D->k1);
+    int E = (int)ceil_div(D->k1, P);
+    P = (int)ceil_div(D->k1, E);
+    int rpp = (int)ceil_div(D->n_out, H);
+    int lb = bitlen(E - 1), rb = bitlen(rpp - 1), eb = lb + rb;
+    int epw = eb <= 21 ? 3 : (eb <= 32 ? 2 : 0);
+    if (epw && rpp <= 65535) {
+      cs_P = P; cs_H = H; cs_E = E; cs_rpp = rpp; cs_lbits = lb; cs_ebits = eb; cs_epw = epw;
+      const int ncta = P * H;
+      std::vector<std::vector<uint32_t>> bucket(ncta);
+      cs_counts.assign((size_t)ncta * n_sub, 0);
+      for (int32_t sv = 0; sv < n_sub; ++sv)
+        for (int32_t i = 0; i < D->n_out; ++i) {
+          uint32_t idx = host_field(codes.data() + (size_t)i * D->row_stride_bytes, sv, w) & m1;
+          int pp = (int)(idx / (uint32_t)E), hh = i / rpp;
+          int cc = pp * H + hh;
+          bucket[cc].push_back(((uint32_t)(i - hh * rpp) << lb) | (idx - (uint32_t)pp * E));
+          cs_counts[(size_t)cc * n_sub + sv] += 1;
+        }
+      cs_start.assign(ncta + 1, 0);
+      const int64_t pad = 8 * epw;       // blocks start on 8-word boundaries (16-byte aligned copies)
+      for (int cc = 0; cc < ncta; ++cc) cs_start[cc + 1] = cs_start[cc] + round_up((int64_t)bucket[cc].size(), pad);
+      cs_words.assign((size_t)(cs_start[ncta] / epw) + 8, 0);
+      cs_wpos.assign(cs_words.size(), 0);
+      for (int cc = 0; cc < ncta; ++cc) {
+        // position of every entry of the bucket, from its per-position counts
+        std::vector<uint16_t> pos(bucket[cc].size());
+        size_t k = 0;
+        for (int32_t sv = 0; sv < n_sub; ++sv)
+          for (int t = 0; t < cs_counts[(size_t)cc * n_sub + sv]; ++t) pos[k++] = (uint16_t)sv;
+        for (k = 0; k < bucket[cc].size(); ++k) {
+          int64_t e = cs_start[cc] + (int64_t)k;
+          cs_words[(size_t)(e / epw)] |= (uint64_t)bucket[cc][k] << ((e % epw) * (epw == 3 ? 21 : 32));
+          if (e % epw == 0) cs_wpos[(size_t)(e / epw)] = pos[k];
+        }
+      }
+    }
+  }
+
   // ---- upload
   vqlin_handle* h = new vqlin_handle();
   memset(h, 0, sizeof *h);
@@ -354,6 +406,17 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
     L.col16 = col16.empty() ? nullptr : up.put<uint16_t>(col16.data(), col16.size() * 2);
   }
   L.tcodes = tcodes.empty() ? nullptr : up.put<uint8_t>(tcodes.data(), tcodes.size());
+  if (!cs_words.empty()) {
+    L.cs_words = up.put<uint64_t>(cs_words.data(), cs_words.size() * 8);
+    L.cs_start = up.put<int64_t>(cs_start.data(), cs_start.size() * 8);
+    L.cs_counts = up.put<uint16_t>(cs_counts.data(), cs_counts.size() * 2);
+    L.cs_wpos = up.put<uint16_t>(cs_wpos.data(), cs_wpos.size() * 2);
+    L.cs_P = cs_P; L.cs_H = cs_H; L.cs_E = cs_E; L.cs_rpp = cs_rpp;
+    L.cs_local_bits = cs_lbits; L.cs_ebits = cs_ebits; L.cs_epw = cs_epw;
+    L.cs_max_words = 0;
+    for (size_t cc = 0; cc + 1 < cs_start.size(); ++cc)
+      L.cs_max_words = std::max<int64_t>(L.cs_max_words, (cs_start[cc + 1] - cs_start[cc]) / cs_epw);
+  }
   L.n_ls = n_ls;
   L.tstride = tstride;
   if (up.st == VQLIN_OK) up.st = cuda_status(cudaStreamSynchronize((cudaStream_t)stream), "create sync");

@@ -235,7 +235,9 @@ cudaError_t launch_gemv_generic(const Layer& L, const void* x, vqlin_dtype xt, i
 cudaError_t launch_gemv(const Layer& L, const void* x, vqlin_dtype xt, int batch, void* y, vqlin_dtype yt,
                         void* ws, size_t ws_bytes, cudaStream_t s) {
   bool handled = false;
-  cudaError_t e = launch_gemv_tc(L, x, xt, batch, y, yt, ws, ws_bytes, s, &handled);
+  cudaError_t e = launch_gemv_cs(L, x, xt, batch, y, yt, ws, ws_bytes, s, &handled);
+  if (e != cudaSuccess || handled) return e;
+  e = launch_gemv_tc(L, x, xt, batch, y, yt, ws, ws_bytes, s, &handled);
   if (e != cudaSuccess || handled) return e;
   return launch_gemv_generic(L, x, xt, batch, y, yt, s);
 }

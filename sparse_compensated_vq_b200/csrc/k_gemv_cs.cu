@@ -1,0 +1,462 @@
+// Codebook-stationary decode GEMV for codebooks too large for one SM's shared
+// memory (K = 65536 entries of d = 8 fp16 = 1 MiB): the fused dequant + GEMV of
+// the VPTQ page ("The dequantization interface", QGemv) reorganised so that
+// every centroid gather is a bank-conflict-free shared-memory load.
+//
+// At create time every sub-vector (row i, position s) of the main block is put
+// in the bucket of thread block (p, h): p = the codebook slice holding its index
+// (slices of E <= 1024 consecutive entries), h = the half of the rows holding i.
+// Inside a bucket the entries are sorted by position s, then row; an entry keeps
+// (row - first row of the half, index - first index of the slice) in a 21-bit
+// slot, three per 64-bit word (32-bit slots, two per word, when it needs more
+// bits).  Per (bucket, position) counts delimit the runs, and every word also
+// records the position of its first entry.
+//
+// A block holds its slice as 8 interleaved copies (entry k of copy c at k*8+c, so
+// the eight lanes of a quarter-warp, which read copies 0..7, always hit eight
+// different bank groups), x' = c (.) x for every position in fp32, and a
+// shared-memory accumulator for the rows of its half.  Its entry words and their
+// start positions arrive by bulk asynchronous copies while it stages the rest.
+// Each lane then takes one word (EPW consecutive entries) at a time: the entries
+// usually share a position, so x'[s] stays in registers; each centroid is one
+// conflict-free 16-byte load; each product is added to its row with a
+// shared-memory atomic.  The block writes its row sums to its own fp32 plane of
+// the caller's workspace, and k_cs_finalize sums the planes per row, applies the
+// row scale and adds the fused sparse correction and the outlier-column block
+// (SCVQ summary step 4; HAS-VQ abstract: sparse entries exact), at full
+// occupancy.  No global atomics: the result is deterministic.  Waits are bounded.
+#include "vqlin_internal.cuh"
+
+namespace vqlin {
+
+namespace csg {
+
+constexpr int WARPS = 16;
+constexpr int THREADS = WARPS * 32;
+constexpr int COPIES = 8;
+constexpr unsigned long long WAIT_NS = 1000000000ull;
+
+__device__ int g_cs_error = 0;
+
+__device__ __forceinline__ uint64_t now_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile("{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+               : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(su32(dst)), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+
+__host__ __device__ inline size_t r16(size_t v) { return (v + 15) & ~size_t(15); }
+
+// Shared-memory layout of a block (byte offsets, every region 16-byte aligned).
+struct Carve {
+  size_t xs, yp, off, bar, words;
+  __host__ __device__ Carve(int E, int n_sub, int NB, int rpp) {
+    xs = r16((size_t)E * COPIES * 16);
+    yp = r16(xs + (size_t)n_sub * NB * 8 * 4);
+    off = r16(yp + (size_t)NB * rpp * 4);
+    bar = r16(off + (size_t)(n_sub + 1) * 4);
+    words = bar + 16;
+  }
+  // entry words then their start positions (u16), for a buffer of `cap` words (cap % 8 == 0)
+  __host__ __device__ size_t wpos(int cap) const { return words + (size_t)cap * 8; }
+  __host__ __device__ size_t total(int cap) const { return wpos(cap) + (size_t)cap * 2; }
+};
+
+struct Args {
+  Layer L;
+  const void* x;
+  vqlin_dtype xt;
+  int batch;
+  float* planes;        // [P][batch][n_out]
+  int words_cap;        // words the shared buffer holds (a multiple of 8)
+};
+
+template <int NB, int EPW>
+__global__ void __launch_bounds__(THREADS, 1) k_gemv_cs(Args a) {
+  constexpr int SLOT = EPW == 3 ? 21 : 32;
+  const Layer& L = a.L;
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int H = L.cs_H, E = L.cs_E, RPP = L.cs_rpp;
+  const int c = blockIdx.x;
+  const int p = c / H, h = c - p * H;
+  const int row0 = h * RPP;
+  const int nrows = min(RPP, L.n_out - row0);
+  const int slice0 = p * E, E_p = max(0, min(E, L.k1 - slice0));
+  const int n_sub = L.n_sub;
+  const int B = a.batch;
+  const Carve cv(E, n_sub, NB, RPP);
+  uint4* cbs = reinterpret_cast<uint4*>(smem);                        // [E][8]
+  float* xs = reinterpret_cast<float*>(smem + cv.xs);                 // [n_sub][NB][8]
+  float* yp = reinterpret_cast<float*>(smem + cv.yp);                 // [NB][RPP]
+  int* off = reinterpret_cast<int*>(smem + cv.off);                   // [n_sub + 1]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + cv.bar);         // mbarrier + abort flag
+  uint64_t* words = reinterpret_cast<uint64_t*>(smem + cv.words);     // [cap]
+  uint16_t* wpos = reinterpret_cast<uint16_t*>(smem + cv.wpos(a.words_cap));   // [cap]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // this block's words: entries [cs_start[c], cs_start[c+1]), a multiple of 8 words
+  const int64_t w_begin = L.cs_start[c] / EPW;
+  const int n_words = (int)((L.cs_start[c + 1] - L.cs_start[c]) / EPW);
+  const bool one_chunk = n_words <= a.words_cap;
+  auto issue_chunk = [&](int w0) {      // thread 0: words [w0, w0 + n) and their positions
+    const int n = min(a.words_cap, n_words - w0);
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(bar)), "r"((uint32_t)(n * 10))
+                 : "memory");
+    bulk_load(words, L.cs_words + w_begin + w0, (uint32_t)(n * 8), su32(bar));
+    bulk_load(wpos, L.cs_wpos + w_begin + w0, (uint32_t)(n * 2), su32(bar));
+  };
+  if (threadIdx.x == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(su32(bar)) : "memory");
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    if (one_chunk && n_words > 0) issue_chunk(0);   // overlaps the staging below
+  }
+  // ---- codebook slice (8 interleaved copies), x' per position, run counts; loads first
+  {
+    const uint4* cb = reinterpret_cast<const uint4*>(L.cb1) + slice0;
+    uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+    const int k0 = threadIdx.x, k1 = threadIdx.x + THREADS;
+    if (k0 < E_p) v0 = __ldg(cb + k0);
+    if (k1 < E_p) v1 = __ldg(cb + k1);
+    const uint16_t* cnt = L.cs_counts + (size_t)c * n_sub;
+    for (int s = threadIdx.x; s < n_sub; s += THREADS) off[s] = cnt[s];
+    with_dtype(a.xt, [&](auto tag) {
+      constexpr int XT = decltype(tag)::value;
+      for (int i = threadIdx.x; i < n_sub * NB; i += THREADS) {
+        const int s = i / NB, b = i - s * NB;
+        int jj[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int q = s * 8 + k;
+          jj[k] = (b < B && q < L.n_main) ? (L.colmap ? L.colmap[q] : q) : -1;
+        }
+        float v[8], cvv[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = jj[k] >= 0 ? ldx<XT>(a.x, (int64_t)b * L.n_in + jj[k]) : 0.f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) cvv[k] = (L.cs && jj[k] >= 0) ? __half2float(L.cs[jj[k]]) : 1.f;
+        float4* dst = reinterpret_cast<float4*>(xs + ((size_t)s * NB + b) * 8);
+        dst[0] = make_float4(v[0] * cvv[0], v[1] * cvv[1], v[2] * cvv[2], v[3] * cvv[3]);
+        dst[1] = make_float4(v[4] * cvv[4], v[5] * cvv[5], v[6] * cvv[6], v[7] * cvv[7]);
+      }
+    });
+    if (k0 < E_p)
+#pragma unroll
+      for (int cc = 0; cc < COPIES; ++cc) cbs[k0 * COPIES + cc] = v0;
+    if (k1 < E_p)
+#pragma unroll
+      for (int cc = 0; cc < COPIES; ++cc) cbs[k1 * COPIES + cc] = v1;
+    for (int k = threadIdx.x + 2 * THREADS; k < E_p; k += THREADS) {   // slices wider than 2*THREADS
+      const uint4 v = __ldg(cb + k);
+#pragma unroll
+      for (int cc = 0; cc < COPIES; ++cc) cbs[k * COPIES + cc] = v;
+    }
+    for (int i = threadIdx.x; i < NB * RPP; i += THREADS) yp[i] = 0.f;
+  }
+  __syncthreads();
+  if (warp == 0) {   // exclusive prefix sum of the counts
+    const int per = (n_sub + 31) / 32;
+    const int s0 = lane * per, s1 = min(n_sub, s0 + per);
+    int local = 0;
+    for (int s = s0; s < s1; ++s) local += off[s];
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - local;
+    for (int s = s0; s < s1; ++s) { const int cs = off[s]; off[s] = run; run += cs; }
+    if (lane == 31) off[n_sub] = incl;
+  }
+  __syncthreads();
+
+  // ---- main loop over the entry words (one chunk when they fit, else chunk by chunk)
+  const uint32_t lmask = (1u << L.cs_local_bits) - 1u;
+  const uint64_t emask = (1ull << L.cs_ebits) - 1ull;
+  const int lbits = L.cs_local_bits;
+  const int n_ent = off[n_sub];                      // real entries (padding is never processed)
+  uint32_t phase = 0;
+  for (int w0 = 0; w0 < n_words; w0 += a.words_cap) {
+    if (!one_chunk) {
+      __syncthreads();
+      if (threadIdx.x == 0) issue_chunk(w0);
+    }
+    if (!one_chunk || w0 == 0) {
+      bool ok = mbar_try(su32(bar), phase);
+      if (!ok) {
+        const uint64_t t0 = now_ns();
+        while (!(ok = mbar_try(su32(bar), phase)))
+          if (now_ns() - t0 > WAIT_NS) { atomicExch(&g_cs_error, 6); *abort_flag = 1; break; }
+      }
+      phase ^= 1u;
+    }
+    __syncthreads();
+    if (*abort_flag) break;
+    const int nw = min(a.words_cap, n_words - w0);
+    const int wb = nw * warp / WARPS, we = nw * (warp + 1) / WARPS;
+    float xr[NB][8];
+    int cur = -1;
+    for (int wi = wb + lane; wi < we; wi += 32) {
+      const int e0 = (w0 + wi) * EPW;                // block-local index of the word's first entry
+      if (e0 >= n_ent) continue;
+      const uint64_t wv = words[wi];
+      int s = wpos[wi];
+      uint32_t ent[EPW];
+      uint4 cen[EPW];
+#pragma unroll
+      for (int u = 0; u < EPW; ++u) {
+        ent[u] = (uint32_t)((wv >> (u * SLOT)) & emask);
+        cen[u] = cbs[(ent[u] & lmask) * COPIES + (lane & (COPIES - 1))];
+      }
+#pragma unroll
+      for (int u = 0; u < EPW; ++u) {
+        const int e = e0 + u;
+        if (e >= n_ent) break;
+        if (u > 0) while (off[s + 1] <= e) ++s;
+        if (s != cur) {
+          cur = s;
+#pragma unroll
+          for (int b = 0; b < NB; ++b) {
+            const float4* xv = reinterpret_cast<const float4*>(xs + ((size_t)s * NB + b) * 8);
+            const float4 x0 = xv[0], x1 = xv[1];
+            xr[b][0] = x0.x; xr[b][1] = x0.y; xr[b][2] = x0.z; xr[b][3] = x0.w;
+            xr[b][4] = x1.x; xr[b][5] = x1.y; xr[b][6] = x1.z; xr[b][7] = x1.w;
+          }
+        }
+        const __half2* h2 = reinterpret_cast<const __half2*>(&cen[u]);
+        float cf[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) { const float2 f2 = __half22float2(h2[k]); cf[2 * k] = f2.x; cf[2 * k + 1] = f2.y; }
+        const int row_l = (int)(ent[u] >> lbits);
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          if (b >= B) continue;
+          float p0 = cf[0] * xr[b][0], p1 = cf[1] * xr[b][1];
+          p0 = fmaf(cf[2], xr[b][2], p0); p1 = fmaf(cf[3], xr[b][3], p1);
+          p0 = fmaf(cf[4], xr[b][4], p0); p1 = fmaf(cf[5], xr[b][5], p1);
+          p0 = fmaf(cf[6], xr[b][6], p0); p1 = fmaf(cf[7], xr[b][7], p1);
+          atomicAdd(yp + (size_t)b * RPP + row_l, p0 + p1);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) {   // a copy still in flight must land before the block exits
+    const uint64_t t0 = now_ns();
+    while (!mbar_try(su32(bar), phase ^ 1u) && now_ns() - t0 < WAIT_NS) {}
+  }
+  // ---- this block's plane: row sums of half h (the row scale is applied at the end)
+  float* plane = a.planes + (size_t)p * B * L.n_out;
+  const bool aborted = *abort_flag;
+  for (int r = threadIdx.x; r < nrows; r += THREADS)
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+      if (b < B) plane[(size_t)b * L.n_out + row0 + r] = aborted ? 0.f : yp[(size_t)b * RPP + r];
+}
+
+// y[b][i] = r_i * (sum_p planes[p][b][i] + outlier block) + sum_e delta_e x[b][col_e].
+// A block takes 32 rows.  The plane sums: 8 groups of 32 threads, group g adds the
+// planes p = g, g+8, ... (all loads issued together, coalesced over the rows), then
+// a shared-memory reduction.  The sparse term: each warp takes four consecutive
+// rows as one range of CSR entries (loads issued eight at a time).  The outlier
+// block: a warp per row, lanes over its sub-vectors.
+template <int NB>
+__global__ void __launch_bounds__(256) k_cs_finalize(Layer L, const float* __restrict__ planes, int P,
+                                                     const void* __restrict__ x, vqlin_dtype xt, int batch,
+                                                     void* __restrict__ y, vqlin_dtype yt) {
+  constexpr int PG = 16;                              // planes per group and round (loads in flight)
+  __shared__ float part[8][NB][32], spv[NB][32], ovv[NB][32];
+  const int i0 = blockIdx.x * 32;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  {
+    const int g = warp, r = lane, i = i0 + r;
+    const size_t stride = (size_t)batch * L.n_out;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      float acc = 0.f;
+      if (b < batch && i < L.n_out) {
+        const float* pp = planes + (size_t)b * L.n_out + i;
+        for (int q0 = g; q0 < P; q0 += 8 * PG) {
+          float v[PG];
+#pragma unroll
+          for (int k = 0; k < PG; ++k) {
+            const int q = q0 + 8 * k;
+            v[k] = q < P ? pp[(size_t)q * stride] : 0.f;
+          }
+#pragma unroll
+          for (int k = 0; k < PG; ++k) acc += v[k];
+        }
+      }
+      part[g][b][r] = acc;
+    }
+  }
+  with_dtype(xt, [&](auto tag) {
+    constexpr int XT = decltype(tag)::value;
+    // sparse term of rows i0 + 4*warp .. +3
+    const int r0 = warp * 4, ib = i0 + r0;
+    float sp[4][NB];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int b = 0; b < NB; ++b) sp[q][b] = 0.f;
+    if (L.nnz > 0 && ib < L.n_out) {
+      const int rows = min(4, L.n_out - ib);
+      int bnd[5];
+#pragma unroll
+      for (int q = 0; q < 5; ++q) bnd[q] = L.row_ptr[ib + min(q, rows)];
+      const int e_end = bnd[4];                      // rows past the last one repeat its end
+      for (int e0 = bnd[0] + lane; e0 < e_end; e0 += 32 * 8) {
+        float dl[8];
+        int jj[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int e = e0 + 32 * u;
+          const bool ok = e < e_end;
+          dl[u] = ok ? L.delta[e] : 0.f;
+          jj[u] = ok ? (L.col16 ? (int)L.col16[e] : L.col[e]) : 0;
+        }
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          if (b >= batch) continue;
+          float xv[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) xv[u] = ldx<XT>(x, (int64_t)b * L.n_in + jj[u]);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int e = e0 + 32 * u;
+            const float pr = dl[u] * xv[u];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (e >= bnd[q] && e < bnd[q + 1]) sp[q][b] += pr;
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sp[q][b] += __shfl_xor_sync(0xffffffffu, sp[q][b], o);
+        if (lane == 0) spv[b][r0 + q] = sp[q][b];
+      }
+    // outlier block: a warp per row (rows warp, warp + 8, ...)
+    for (int rr = warp; rr < 32; rr += 8) {
+      const int i = i0 + rr;
+      float ov[NB];
+#pragma unroll
+      for (int b = 0; b < NB; ++b) ov[b] = 0.f;
+      if (i < L.n_out) {
+        for (int so = lane; so < L.n_sub_o; so += 32) {
+          const uint32_t f = read_field(L.codes_o + (int64_t)i * L.stride_o, so, L.bits_o);
+          const uint4 u = __ldg(reinterpret_cast<const uint4*>(L.cbo) + f);
+          const __half* hv = reinterpret_cast<const __half*>(&u);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int pcol = so * 8 + k;
+            if (pcol >= L.n_ocols) break;
+            const int j = L.colmap[L.n_main + pcol];
+            const float cj = L.cs ? __half2float(L.cs[j]) : 1.f;
+            const float ck = __half2float(hv[k]);
+#pragma unroll
+            for (int b = 0; b < NB; ++b)
+              if (b < batch) ov[b] = fmaf(ck, cj * ldx<XT>(x, (int64_t)b * L.n_in + j), ov[b]);
+          }
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ov[b] += __shfl_xor_sync(0xffffffffu, ov[b], o);
+        if (lane == 0) ovv[b][rr] = ov[b];
+      }
+    }
+  });
+  __syncthreads();
+  {
+    const int b = t >> 5, r = t & 31;
+    const int i = i0 + r;
+    if (b < NB && b < batch && i < L.n_out) {
+      float body = 0.f;
+#pragma unroll
+      for (int g = 0; g < 8; ++g) body += part[g][b][r];
+      const float rsc = L.rs ? __half2float(L.rs[i]) : 1.f;
+      store_from_float(y, yt, (int64_t)b * L.n_out + i, fmaf(rsc, body + ovv[b][r], spv[b][r]));
+    }
+  }
+}
+
+template <int NB, int EPW>
+static cudaError_t launch_cfg(const Args& a, size_t smem, cudaStream_t s) {
+  auto k = k_gemv_cs<NB, EPW>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k<<<a.L.cs_P * a.L.cs_H, THREADS, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace csg
+
+int read_and_clear_cs_error() {
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, csg::g_cs_error, sizeof v) != cudaSuccess) return -1;
+  if (v) cudaMemcpyToSymbol(csg::g_cs_error, &zero, sizeof zero);
+  return v;
+}
+
+size_t gemv_cs_workspace_bytes(const Layer& L, int batch) {
+  if (!L.cs_words || batch > 4) return 0;
+  return ((size_t)L.cs_P * batch * L.n_out * 4 + 255) & ~size_t(255);
+}
+
+cudaError_t launch_gemv_cs(const Layer& L, const void* x, vqlin_dtype xt, int batch, void* y, vqlin_dtype yt,
+                           void* ws, size_t ws_bytes, cudaStream_t s, bool* handled) {
+  using namespace csg;
+  *handled = false;
+  if (!L.cs_words || batch < 1 || batch > 4) return cudaSuccess;
+  const size_t need = gemv_cs_workspace_bytes(L, batch);
+  if (!ws || ws_bytes < need) return cudaSuccess;
+  const int NB = batch == 1 ? 1 : (batch == 2 ? 2 : 4);
+  const size_t smem_max = 227 * 1024;
+  const Carve cv(L.cs_E, L.n_sub, NB, L.cs_rpp);
+  if (cv.total(64) > smem_max) return cudaSuccess;
+  Args a;
+  a.L = L; a.x = x; a.xt = xt; a.batch = batch; a.planes = reinterpret_cast<float*>(ws);
+  int cap = (int)(((smem_max - cv.words) / 10) & ~7ll);      // 8 + 2 bytes per word, whole groups of 8
+  const int need_words = (int)((L.cs_max_words + 7) & ~7ll);
+  if (need_words < cap) cap = need_words;
+  a.words_cap = cap < 8 ? 8 : cap;
+  const size_t smem = cv.total(a.words_cap);
+  cudaError_t e;
+  if (L.cs_epw == 3) {
+    if (NB == 1) e = launch_cfg<1, 3>(a, smem, s);
+    else if (NB == 2) e = launch_cfg<2, 3>(a, smem, s);
+    else e = launch_cfg<4, 3>(a, smem, s);
+  } else {
+    if (NB == 1) e = launch_cfg<1, 2>(a, smem, s);
+    else if (NB == 2) e = launch_cfg<2, 2>(a, smem, s);
+    else e = launch_cfg<4, 2>(a, smem, s);
+  }
+  if (e != cudaSuccess) return e;
+  const int blocks = (L.n_out + 31) / 32;
+  if (NB == 1) k_cs_finalize<1><<<blocks, 256, 0, s>>>(L, a.planes, L.cs_P, x, xt, batch, y, yt);
+  else if (NB == 2) k_cs_finalize<2><<<blocks, 256, 0, s>>>(L, a.planes, L.cs_P, x, xt, batch, y, yt);
+  else k_cs_finalize<4><<<blocks, 256, 0, s>>>(L, a.planes, L.cs_P, x, xt, batch, y, yt);
+  e = cudaGetLastError();
+  *handled = (e == cudaSuccess);
+  return e;
+}
+
+}  // namespace vqlin

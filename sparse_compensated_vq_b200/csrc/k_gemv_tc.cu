@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
           int bb, part_lo;
-          if (NT == 1) { bb = g & 3; part_lo = g >> 2; }
+          if constexpr (NT == 1) { bb = g & 3; part_lo = g >> 2; }
           else { part_lo = n / (NT / 2); bb = (n % (NT / 2)) * 8 + g; }
           uint4 v = make_uint4(0, 0, 0, 0);
           if (bb < B) v = *reinterpret_cast<const uint4*>((part_lo ? xl : xh) + (size_t)bb * a.xs_cols + col);
@@ -589,7 +589,7 @@ __global__ void __launch_bounds__(THREADS, 2) k_gemv_wt(Args a) {
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
           int bb, part_lo;
-          if (NT == 1) { bb = g & 3; part_lo = g >> 2; }
+          if constexpr (NT == 1) { bb = g & 3; part_lo = g >> 2; }
           else { part_lo = n / (NT / 2); bb = (n % (NT / 2)) * 8 + g; }
           uint4 bv = make_uint4(0, 0, 0, 0);
           if (bb < B) bv = *reinterpret_cast<const uint4*>((part_lo ? xl : xh) + (size_t)bb * a.xs_cols + col);
@@ -703,7 +703,9 @@ bool tc_supported(const Layer& L) {
 }
 
 size_t gemv_workspace_bytes(const Layer& L, int batch) {
-  return ((size_t)batch * L.n_out * 4 + 255) & ~size_t(255);
+  const size_t acc = ((size_t)batch * L.n_out * 4 + 255) & ~size_t(255);
+  const size_t cs = gemv_cs_workspace_bytes(L, batch);
+  return acc > cs ? acc : cs;
 }
 
 // Plan and launch.  acc_ws: caller workspace for split accumulation (may be null).

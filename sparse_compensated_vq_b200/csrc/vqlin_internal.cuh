@@ -40,6 +40,18 @@ struct Layer {
   const uint8_t* tcodes;
   int32_t n_ls;                         // layout slabs per row
   int64_t tstride;                      // bytes per row = n_ls * 8 * w
+  // Codebook-stationary layout (large single-stage codebooks, d = 8; null otherwise):
+  // block c = p * cs_H + h owns codebook slice p (entries [p*cs_E, (p+1)*cs_E)) and row half h
+  // (rows [h*cs_rpp, ...)); its entries (row - h*cs_rpp) << cs_local_bits | (index - p*cs_E),
+  // cs_ebits wide, cs_epw per 64-bit word in slots of 21 (cs_epw = 3) or 32 bits (cs_epw = 2),
+  // sorted by position then row, start at entry
+  // cs_start[c] (a multiple of 8*cs_epw); cs_counts[c*n_sub + s] entries at position s.
+  const uint64_t* cs_words;
+  const int64_t* cs_start;              // [cs_P*cs_H + 1]
+  const uint16_t* cs_counts;            // [cs_P*cs_H][n_sub]
+  const uint16_t* cs_wpos;              // position of the first entry of every word
+  int32_t cs_P, cs_H, cs_E, cs_rpp, cs_local_bits, cs_ebits, cs_epw;
+  int64_t cs_max_words;                 // largest block's word count
 };
 
 // Last-error plumbing (thread-local detail string).
@@ -59,6 +71,10 @@ cudaError_t launch_gemv_generic(const Layer& L, const void* x, vqlin_dtype xt, i
                                 cudaStream_t s);
 cudaError_t launch_convert_to_f16(const void* X, vqlin_dtype xt, int64_t n, __half* out, cudaStream_t s);
 int read_and_clear_device_error();
+int read_and_clear_cs_error();
+size_t gemv_cs_workspace_bytes(const Layer& L, int batch);
+cudaError_t launch_gemv_cs(const Layer& L, const void* x, vqlin_dtype xt, int batch, void* y, vqlin_dtype yt,
+                           void* ws, size_t ws_bytes, cudaStream_t s, bool* handled);
 cudaError_t launch_gemm_f16(const __half* A, const __half* W, int64_t M, int N, int K, void* Y, vqlin_dtype yt,
                             cudaStream_t s);
 
@@ -68,6 +84,29 @@ __device__ __forceinline__ float load_as_float(const void* p, vqlin_dtype t, int
   unsigned short h = __ldg(reinterpret_cast<const unsigned short*>(p) + i);
   if (t == VQLIN_F16) return __half2float(__ushort_as_half(h));
   return __bfloat162float(__ushort_as_bfloat16(h));
+}
+
+// Same with the dtype fixed at compile time, so loads in a loop can be issued together.
+template <int XT>
+__device__ __forceinline__ float ldx(const void* p, int64_t i) {
+  if constexpr (XT == VQLIN_F32) {
+    return __ldg(reinterpret_cast<const float*>(p) + i);
+  } else {
+    unsigned short h = __ldg(reinterpret_cast<const unsigned short*>(p) + i);
+    if constexpr (XT == VQLIN_F16) return __half2float(__ushort_as_half(h));
+    else return __bfloat162float(__ushort_as_bfloat16(h));
+  }
+}
+
+template <int V>
+struct dtype_tag { static constexpr int value = V; };
+
+// Calls f(dtype_tag<XT>{}) with XT the runtime dtype t (a uniform branch outside the caller's loops).
+template <class F>
+__device__ __forceinline__ void with_dtype(vqlin_dtype t, F&& f) {
+  if (t == VQLIN_F32) f(dtype_tag<VQLIN_F32>{});
+  else if (t == VQLIN_F16) f(dtype_tag<VQLIN_F16>{});
+  else f(dtype_tag<VQLIN_BF16>{});
 }
 
 __device__ __forceinline__ void store_from_float(void* p, vqlin_dtype t, int64_t i, float v) {
@@ -100,6 +139,6 @@ struct vqlin_handle {
   // info
   vqlin_info info;
   // allocations to free
-  void* allocs[16];
+  void* allocs[24];
   int n_allocs;
 };

@@ -361,3 +361,49 @@ def test_gemv_ws_errors(vq):
     assert vq.vqlin_gemv_ws(m.handle, x.data_ptr(), vq.VQLIN_F16, 2, y.data_ptr(), vq.VQLIN_F16, ws.data_ptr() + 16, need, None) == vq.VQLIN_ERR_WORKSPACE
     assert vq.vqlin_gemv_ws(m.handle, x.data_ptr(), vq.VQLIN_F16, 2, y.data_ptr(), vq.VQLIN_F16, ws.data_ptr(), need, None) == vq.VQLIN_OK
     torch.cuda.synchronize()
+
+
+# ------------------------------------------------------------------ codebook-stationary path (large K, caller workspace)
+def cs_layers():
+    rng = np.random.default_rng(8080)
+    out = [
+        synth.random_layer(rng, 300, 1024, 8, 65536, 16, col_scale=True, nnz=500, name="cs_h1"),
+        synth.random_layer(rng, 2100, 520, 8, 20000, 15, nnz=300, n_ocols=8, ko=64, bits_o=6, name="cs_h2_oddk"),
+    ]
+    # skewed: every index in the first slice -> one block's entry stream is far larger than its buffer
+    n_out, n_in = 2048, 2048
+    fields = rng.integers(0, 600, size=(n_out, n_in // 8)).astype(np.uint32)
+    L = synth.random_layer(rng, n_out, n_in, 8, 65536, 16, col_scale=True, nnz=200, name="cs_skewed")
+    L.codes = synth.pack_fields(fields, 16)
+    L.fields = fields
+    out.append(L)
+    return out
+
+
+CS = cs_layers()
+
+
+@pytest.mark.parametrize("t", range(len(CS)))
+@pytest.mark.parametrize("batch", [1, 2, 3, 4])
+def test_gemv_codebook_stationary(vq, t, batch):
+    import torch
+    L = CS[t]
+    rng = np.random.default_rng(60 + 10 * t + batch)
+    xb = synth.activations(rng, batch, L.n_in, "f16")
+    m = vq.VQLinear(L)
+    x = G.torch_x(xb, "f16")
+    y = m.gemv_ws(x, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert vq.device_error() == 0
+    G.assert_close(G.to_f64(y), oracle.gemv_f64(L, synth.bits_to_f64(xb, "f16")), "f32", "%s B=%d" % (L.name, batch))
+
+
+def test_gemv_codebook_stationary_full_qproj(vq):
+    import torch
+    L, xb = G.workload("qproj")
+    m = vq.VQLinear(L)
+    for batch in (1, 4):
+        x = G.torch_x(xb[:batch], "f16")
+        y = m.gemv_ws(x, out_dtype=torch.float16)
+        torch.cuda.synchronize()
+        G.assert_close(G.to_f64(y), oracle.gemv_f64(L, synth.bits_to_f64(xb[:batch], "f16")), "f16", "qproj cs B=%d" % batch)
