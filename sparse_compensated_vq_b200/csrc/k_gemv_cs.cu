@@ -116,13 +116,16 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_cs(Args a) {
     bulk_load(words, L.cs_words + w_begin + w0, (uint32_t)(n * 8), su32(bar));
     bulk_load(wpos, L.cs_wpos + w_begin + w0, (uint32_t)(n * 2), su32(bar));
   };
+  // the finalize kernel may start now: its sparse/outlier work does not read this grid's output
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (threadIdx.x == 0) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(su32(bar)) : "memory");
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     if (one_chunk && n_words > 0) issue_chunk(0);   // overlaps the staging below
   }
-  // ---- codebook slice (8 interleaved copies), x' per position, run counts; loads first
+  // ---- codebook slice (8 interleaved copies), x' per position, run counts; every
+  //      global load of this phase is issued before any of its values is used
   {
     const uint4* cb = reinterpret_cast<const uint4*>(L.cb1) + slice0;
     uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
@@ -130,27 +133,51 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_cs(Args a) {
     if (k0 < E_p) v0 = __ldg(cb + k0);
     if (k1 < E_p) v1 = __ldg(cb + k1);
     const uint16_t* cnt = L.cs_counts + (size_t)c * n_sub;
-    for (int s = threadIdx.x; s < n_sub; s += THREADS) off[s] = cnt[s];
+    int cnt0 = threadIdx.x < n_sub ? cnt[threadIdx.x] : 0;
+    // x' for (position s, batch b), one item per thread per round: 16-byte loads of x and c when
+    // the main columns are contiguous and 8-aligned, else eight clamped scalar loads
+    const bool vec = !L.colmap && a.xt != VQLIN_F32 && (L.n_in & 7) == 0;
     with_dtype(a.xt, [&](auto tag) {
       constexpr int XT = decltype(tag)::value;
       for (int i = threadIdx.x; i < n_sub * NB; i += THREADS) {
         const int s = i / NB, b = i - s * NB;
-        int jj[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int q = s * 8 + k;
-          jj[k] = (b < B && q < L.n_main) ? (L.colmap ? L.colmap[q] : q) : -1;
-        }
+        const int q0 = s * 8;
         float v[8], cvv[8];
+        if (XT != VQLIN_F32 && vec && b < B && q0 + 8 <= L.n_main) {
+          const uint4 u = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const unsigned short*>(a.x) +
+                                                              (int64_t)b * L.n_in + q0));
+          uint4 cu = make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);   // fp16 ones
+          if (L.cs) cu = __ldg(reinterpret_cast<const uint4*>(L.cs + q0));
+          const unsigned short* hs = reinterpret_cast<const unsigned short*>(&u);
+          const __half* ch = reinterpret_cast<const __half*>(&cu);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) v[k] = jj[k] >= 0 ? ldx<XT>(a.x, (int64_t)b * L.n_in + jj[k]) : 0.f;
+          for (int k = 0; k < 8; ++k) {
+            v[k] = XT == VQLIN_F16 ? __half2float(__ushort_as_half(hs[k])) : __bfloat162float(__ushort_as_bfloat16(hs[k]));
+            cvv[k] = __half2float(ch[k]);
+          }
+        } else {
+          int jj[8];
+          bool ok[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) cvv[k] = (L.cs && jj[k] >= 0) ? __half2float(L.cs[jj[k]]) : 1.f;
+          for (int k = 0; k < 8; ++k) {
+            const int q = q0 + k;
+            ok[k] = b < B && q < L.n_main;
+            jj[k] = ok[k] ? (L.colmap ? L.colmap[q] : q) : 0;
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k) v[k] = ldx<XT>(a.x, (int64_t)(b < B ? b : 0) * L.n_in + jj[k]);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) cvv[k] = L.cs ? __half2float(L.cs[jj[k]]) : 1.f;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) if (!ok[k]) v[k] = 0.f;
+        }
         float4* dst = reinterpret_cast<float4*>(xs + ((size_t)s * NB + b) * 8);
         dst[0] = make_float4(v[0] * cvv[0], v[1] * cvv[1], v[2] * cvv[2], v[3] * cvv[3]);
         dst[1] = make_float4(v[4] * cvv[4], v[5] * cvv[5], v[6] * cvv[6], v[7] * cvv[7]);
       }
     });
+    if (threadIdx.x < n_sub) off[threadIdx.x] = cnt0;
+    for (int s2 = threadIdx.x + THREADS; s2 < n_sub; s2 += THREADS) off[s2] = cnt[s2];
     if (k0 < E_p)
 #pragma unroll
       for (int cc = 0; cc < COPIES; ++cc) cbs[k0 * COPIES + cc] = v0;
@@ -267,11 +294,13 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_cs(Args a) {
 }
 
 // y[b][i] = r_i * (sum_p planes[p][b][i] + outlier block) + sum_e delta_e x[b][col_e].
-// A block takes 32 rows.  The plane sums: 8 groups of 32 threads, group g adds the
-// planes p = g, g+8, ... (all loads issued together, coalesced over the rows), then
-// a shared-memory reduction.  The sparse term: each warp takes four consecutive
-// rows as one range of CSR entries (loads issued eight at a time).  The outlier
-// block: a warp per row, lanes over its sub-vectors.
+// A block takes 32 rows.  It is launched as a programmatic dependent of the
+// codebook-stationary grid, so it first computes the terms that do not need that
+// grid's output (sparse term: each warp takes four consecutive rows as one range
+// of CSR entries, loads issued eight at a time; outlier block: a warp per row),
+// then waits for the grid and sums the planes: 8 groups of 32 threads, group g
+// adds the planes p = g, g+8, ... (loads issued together, coalesced over the
+// rows), then a shared-memory reduction.
 template <int NB>
 __global__ void __launch_bounds__(256) k_cs_finalize(Layer L, const float* __restrict__ planes, int P,
                                                      const void* __restrict__ x, vqlin_dtype xt, int batch,
@@ -280,28 +309,6 @@ __global__ void __launch_bounds__(256) k_cs_finalize(Layer L, const float* __res
   __shared__ float part[8][NB][32], spv[NB][32], ovv[NB][32];
   const int i0 = blockIdx.x * 32;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  {
-    const int g = warp, r = lane, i = i0 + r;
-    const size_t stride = (size_t)batch * L.n_out;
-#pragma unroll
-    for (int b = 0; b < NB; ++b) {
-      float acc = 0.f;
-      if (b < batch && i < L.n_out) {
-        const float* pp = planes + (size_t)b * L.n_out + i;
-        for (int q0 = g; q0 < P; q0 += 8 * PG) {
-          float v[PG];
-#pragma unroll
-          for (int k = 0; k < PG; ++k) {
-            const int q = q0 + 8 * k;
-            v[k] = q < P ? pp[(size_t)q * stride] : 0.f;
-          }
-#pragma unroll
-          for (int k = 0; k < PG; ++k) acc += v[k];
-        }
-      }
-      part[g][b][r] = acc;
-    }
-  }
   with_dtype(xt, [&](auto tag) {
     constexpr int XT = decltype(tag)::value;
     // sparse term of rows i0 + 4*warp .. +3
@@ -384,6 +391,30 @@ __global__ void __launch_bounds__(256) k_cs_finalize(Layer L, const float* __res
       }
     }
   });
+  // the planes are written by the preceding codebook-stationary grid
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  {
+    const int g = warp, r = lane, i = i0 + r;
+    const size_t stride = (size_t)batch * L.n_out;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      float acc = 0.f;
+      if (b < batch && i < L.n_out) {
+        const float* pp = planes + (size_t)b * L.n_out + i;
+        for (int q0 = g; q0 < P; q0 += 8 * PG) {
+          float v[PG];
+#pragma unroll
+          for (int k = 0; k < PG; ++k) {
+            const int q = q0 + 8 * k;
+            v[k] = q < P ? pp[(size_t)q * stride] : 0.f;
+          }
+#pragma unroll
+          for (int k = 0; k < PG; ++k) acc += v[k];
+        }
+      }
+      part[g][b][r] = acc;
+    }
+  }
   __syncthreads();
   {
     const int b = t >> 5, r = t & 31;
@@ -450,11 +481,22 @@ cudaError_t launch_gemv_cs(const Layer& L, const void* x, vqlin_dtype xt, int ba
     else e = launch_cfg<4, 2>(a, smem, s);
   }
   if (e != cudaSuccess) return e;
-  const int blocks = (L.n_out + 31) / 32;
-  if (NB == 1) k_cs_finalize<1><<<blocks, 256, 0, s>>>(L, a.planes, L.cs_P, x, xt, batch, y, yt);
-  else if (NB == 2) k_cs_finalize<2><<<blocks, 256, 0, s>>>(L, a.planes, L.cs_P, x, xt, batch, y, yt);
-  else k_cs_finalize<4><<<blocks, 256, 0, s>>>(L, a.planes, L.cs_P, x, xt, batch, y, yt);
-  e = cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3((L.n_out + 31) / 32);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const float* planes = a.planes;
+  const int P = L.cs_P;
+  if (NB == 1) e = cudaLaunchKernelEx(&cfg, k_cs_finalize<1>, L, planes, P, x, xt, batch, y, yt);
+  else if (NB == 2) e = cudaLaunchKernelEx(&cfg, k_cs_finalize<2>, L, planes, P, x, xt, batch, y, yt);
+  else e = cudaLaunchKernelEx(&cfg, k_cs_finalize<4>, L, planes, P, x, xt, batch, y, yt);
+  if (e == cudaSuccess) e = cudaGetLastError();
   *handled = (e == cudaSuccess);
   return e;
 }
