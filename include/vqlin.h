@@ -251,6 +251,15 @@ vqlin_status vqlin_unpack_indices(const vqlin_handle* h, int32_t which, uint32_t
  */
 vqlin_status vqlin_device_error(int32_t* code);
 
+/*
+ * Number of kernels this library has enqueued in this process so far, over
+ * every device, stream and thread (a launch recorded into a CUDA graph counts
+ * once, when it is recorded).  Library copies and memsets are not counted.
+ * Take the difference around a call to learn how many kernels it launched.
+ * No counterpart on the pages.
+ */
+uint64_t vqlin_kernel_launches(void);
+
 const char* vqlin_status_string(vqlin_status s);
 const char* vqlin_last_error(void);
 int32_t vqlin_abi_version(void);

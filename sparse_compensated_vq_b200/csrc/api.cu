@@ -2,6 +2,7 @@
 // bit accounting, errors and dispatch.  The arithmetic of every call runs in
 // the kernels of k_*.cu; create-time preparation runs here.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -14,6 +15,9 @@
 namespace vqlin {
 
 static thread_local std::string g_err;
+static std::atomic<uint64_t> g_kernel_launches{0};
+
+void note_launches(int n) { g_kernel_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
 void set_error(const char* fmt, ...) {
   char buf[512];
@@ -122,6 +126,8 @@ vqlin_status vqlin_device_error(int32_t* code) {
   return VQLIN_OK;
 }
 int32_t vqlin_abi_version(void) { return VQLIN_ABI_VERSION; }
+
+uint64_t vqlin_kernel_launches(void) { return vqlin::g_kernel_launches.load(std::memory_order_relaxed); }
 
 vqlin_status vqlin_destroy(vqlin_handle* h) {
   if (!h) return VQLIN_OK;
@@ -330,50 +336,52 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
   // codebook-stationary layout for large single-stage codebooks (see vqlin_internal.cuh)
   std::vector<uint64_t> cs_words;
   std::vector<int64_t> cs_start;
-  std::vector<uint16_t> cs_counts, cs_wpos;
+  std::vector<uint16_t> cs_wpos;
   int32_t cs_P = 0, cs_H = 0, cs_E = 0, cs_rpp = 0, cs_lbits = 0, cs_ebits = 0, cs_epw = 0;
-  if (d == 8 && D->k2 == 0 && D->k1 > 10240 && n_sub > 0) {
+  if (d == 8 && D->k2 == 0 && D->k1 > 10240 && n_sub > 0 && n_sub <= 65536) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     auto bitlen = [](int64_t v) { int b = 0; while ((1ll << b) <= v) ++b; return b < 1 ? 1 : b; };
     int H = D->n_out >= 2048 ? 2 : 1;
-    int P = (int)std::max<int64_t>(ceil_div(D->k1, 1024), std::max(1, sms / H));
+    int P = (int)std::max<int64_t>(ceil_div(D->k1, 1023), std::max(1, sms / H));
     P = std::min(P, D->k1);
     int E = (int)ceil_div(D->k1, P);
     P = (int)ceil_div(D->k1, E);
     int rpp = (int)ceil_div(D->n_out, H);
-    int lb = bitlen(E - 1), rb = bitlen(rpp - 1), eb = lb + rb;
+    int lb = bitlen(E), rb = bitlen(rpp - 1), eb = lb + rb;     // local indices 0..E (E = null entry)
     int epw = eb <= 21 ? 3 : (eb <= 32 ? 2 : 0);
     if (epw && rpp <= 65535) {
       cs_P = P; cs_H = H; cs_E = E; cs_rpp = rpp; cs_lbits = lb; cs_ebits = eb; cs_epw = epw;
       const int ncta = P * H;
-      std::vector<std::vector<uint32_t>> bucket(ncta);
-      cs_counts.assign((size_t)ncta * n_sub, 0);
-      for (int32_t sv = 0; sv < n_sub; ++sv)
+      const int slot = epw == 3 ? 21 : 32;
+      const uint32_t null_entry = (uint32_t)E;                  // row 0, zero centroid
+      std::vector<std::vector<uint64_t>> bw(ncta);              // words of every block
+      std::vector<std::vector<uint16_t>> bp(ncta);              // their positions
+      std::vector<int> fill(ncta, 0);                           // entries in the block's open word
+      auto put = [&](int cc, uint32_t ent, int32_t sv) {
+        if (fill[cc] == 0) { bw[cc].push_back(0); bp[cc].push_back((uint16_t)sv); }
+        bw[cc].back() |= (uint64_t)ent << (fill[cc] * slot);
+        fill[cc] = (fill[cc] + 1) % epw;
+      };
+      for (int32_t sv = 0; sv < n_sub; ++sv) {
         for (int32_t i = 0; i < D->n_out; ++i) {
           uint32_t idx = host_field(codes.data() + (size_t)i * D->row_stride_bytes, sv, w) & m1;
           int pp = (int)(idx / (uint32_t)E), hh = i / rpp;
-          int cc = pp * H + hh;
-          bucket[cc].push_back(((uint32_t)(i - hh * rpp) << lb) | (idx - (uint32_t)pp * E));
-          cs_counts[(size_t)cc * n_sub + sv] += 1;
+          put(pp * H + hh, ((uint32_t)(i - hh * rpp) << lb) | (idx - (uint32_t)pp * E), sv);
         }
+        for (int cc = 0; cc < ncta; ++cc)   // close the run of position sv
+          while (fill[cc] != 0) put(cc, null_entry, sv);
+      }
+      uint64_t null_word = 0;
+      for (int u = 0; u < epw; ++u) null_word |= (uint64_t)null_entry << (u * slot);
       cs_start.assign(ncta + 1, 0);
-      const int64_t pad = 8 * epw;       // blocks start on 8-word boundaries (16-byte aligned copies)
-      for (int cc = 0; cc < ncta; ++cc) cs_start[cc + 1] = cs_start[cc] + round_up((int64_t)bucket[cc].size(), pad);
-      cs_words.assign((size_t)(cs_start[ncta] / epw) + 8, 0);
+      for (int cc = 0; cc < ncta; ++cc) cs_start[cc + 1] = cs_start[cc] + round_up((int64_t)bw[cc].size(), 8);
+      cs_words.assign((size_t)cs_start[ncta], null_word);
       cs_wpos.assign(cs_words.size(), 0);
       for (int cc = 0; cc < ncta; ++cc) {
-        // position of every entry of the bucket, from its per-position counts
-        std::vector<uint16_t> pos(bucket[cc].size());
-        size_t k = 0;
-        for (int32_t sv = 0; sv < n_sub; ++sv)
-          for (int t = 0; t < cs_counts[(size_t)cc * n_sub + sv]; ++t) pos[k++] = (uint16_t)sv;
-        for (k = 0; k < bucket[cc].size(); ++k) {
-          int64_t e = cs_start[cc] + (int64_t)k;
-          cs_words[(size_t)(e / epw)] |= (uint64_t)bucket[cc][k] << ((e % epw) * (epw == 3 ? 21 : 32));
-          if (e % epw == 0) cs_wpos[(size_t)(e / epw)] = pos[k];
-        }
+        std::copy(bw[cc].begin(), bw[cc].end(), cs_words.begin() + cs_start[cc]);
+        std::copy(bp[cc].begin(), bp[cc].end(), cs_wpos.begin() + cs_start[cc]);
       }
     }
   }
@@ -409,13 +417,12 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
   if (!cs_words.empty()) {
     L.cs_words = up.put<uint64_t>(cs_words.data(), cs_words.size() * 8);
     L.cs_start = up.put<int64_t>(cs_start.data(), cs_start.size() * 8);
-    L.cs_counts = up.put<uint16_t>(cs_counts.data(), cs_counts.size() * 2);
     L.cs_wpos = up.put<uint16_t>(cs_wpos.data(), cs_wpos.size() * 2);
     L.cs_P = cs_P; L.cs_H = cs_H; L.cs_E = cs_E; L.cs_rpp = cs_rpp;
     L.cs_local_bits = cs_lbits; L.cs_ebits = cs_ebits; L.cs_epw = cs_epw;
     L.cs_max_words = 0;
     for (size_t cc = 0; cc + 1 < cs_start.size(); ++cc)
-      L.cs_max_words = std::max<int64_t>(L.cs_max_words, (cs_start[cc + 1] - cs_start[cc]) / cs_epw);
+      L.cs_max_words = std::max<int64_t>(L.cs_max_words, cs_start[cc + 1] - cs_start[cc]);
   }
   L.n_ls = n_ls;
   L.tstride = tstride;

@@ -128,6 +128,7 @@ static int grid_for(int64_t work, int threads) {
 cudaError_t launch_unpack(const Layer& L, int which, uint32_t* out, cudaStream_t s) {
   int n_fields = which ? L.n_sub_o : L.n_sub;
   if (n_fields == 0) return cudaSuccess;
+  note_launches(1);
   k_unpack<<<grid_for((int64_t)L.n_out * n_fields, 256), 256, 0, s>>>(
       which ? L.codes_o : L.codes, which ? L.stride_o : L.stride, L.n_out, n_fields, which ? L.bits_o : L.w, out);
   return cudaGetLastError();
@@ -136,12 +137,14 @@ cudaError_t launch_unpack(const Layer& L, int which, uint32_t* out, cudaStream_t
 cudaError_t launch_dequant(const Layer& L, __half* W, int64_t ldw, cudaStream_t s) {
   int64_t work = (int64_t)L.n_out * (L.n_sub + L.n_sub_o);
   if (work > 0) {
+    note_launches(1);
     if (L.d == 8) k_dequant_body<8><<<grid_for(work, 256), 256, 0, s>>>(L, W, ldw);
     else k_dequant_body<4><<<grid_for(work, 256), 256, 0, s>>>(L, W, ldw);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   if (L.nnz > 0) {
+    note_launches(1);
     k_dequant_sparse<<<grid_for((int64_t)L.n_out * 32, 256), 256, 0, s>>>(L, W, ldw);
     return cudaGetLastError();
   }
@@ -149,6 +152,7 @@ cudaError_t launch_dequant(const Layer& L, __half* W, int64_t ldw, cudaStream_t 
 }
 
 cudaError_t launch_convert_to_f16(const void* X, vqlin_dtype xt, int64_t n, __half* out, cudaStream_t s) {
+  note_launches(1);
   k_convert_f16<<<grid_for(n, 256), 256, 0, s>>>(reinterpret_cast<const unsigned short*>(X), xt, n, out);
   return cudaGetLastError();
 }

@@ -303,6 +303,7 @@ cudaError_t launch_gemm_f16(const __half* A, const __half* W, int64_t M, int N, 
     attr = true;
   }
   dim3 grid((N + tc::BN - 1) / tc::BN, (unsigned)((M + tc::BM - 1) / tc::BM));
+  note_launches(1);
   tc::k_gemm_tc<<<grid, tc::THREADS, tc::SMEM_BYTES, s>>>(ma, mw, M, N, K, Y, yt);
   return cudaGetLastError();
 }

@@ -207,11 +207,13 @@ static cudaError_t launch_generic_nb(const Layer& L, const void* x, vqlin_dtype 
     auto k = k_gemv_generic<D, NB, true>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    note_launches(1);
     k<<<grid, kThreads, smem, s>>>(L, x, xt, batch, y, yt, chunk);
   } else {
     auto k = k_gemv_generic<D, NB, false>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    note_launches(1);
     k<<<grid, kThreads, smem, s>>>(L, x, xt, batch, y, yt, chunk);
   }
   return cudaGetLastError();

@@ -5,26 +5,27 @@
 //
 // At create time every sub-vector (row i, position s) of the main block is put
 // in the bucket of thread block (p, h): p = the codebook slice holding its index
-// (slices of E <= 1024 consecutive entries), h = the half of the rows holding i.
+// (slices of E < 1024 consecutive entries), h = the half of the rows holding i.
 // Inside a bucket the entries are sorted by position s, then row; an entry keeps
 // (row - first row of the half, index - first index of the slice) in a 21-bit
 // slot, three per 64-bit word (32-bit slots, two per word, when it needs more
-// bits).  Per (bucket, position) counts delimit the runs, and every word also
-// records the position of its first entry.
+// bits).  Each run of one position is padded to whole words with a null entry
+// (local index E, a zero centroid), so every word carries one position, which is
+// stored beside it.
 //
 // A block holds its slice as 8 interleaved copies (entry k of copy c at k*8+c, so
 // the eight lanes of a quarter-warp, which read copies 0..7, always hit eight
 // different bank groups), x' = c (.) x for every position in fp32, and a
 // shared-memory accumulator for the rows of its half.  Its entry words and their
-// start positions arrive by bulk asynchronous copies while it stages the rest.
-// Each lane then takes one word (EPW consecutive entries) at a time: the entries
-// usually share a position, so x'[s] stays in registers; each centroid is one
-// conflict-free 16-byte load; each product is added to its row with a
-// shared-memory atomic.  The block writes its row sums to its own fp32 plane of
-// the caller's workspace, and k_cs_finalize sums the planes per row, applies the
-// row scale and adds the fused sparse correction and the outlier-column block
-// (SCVQ summary step 4; HAS-VQ abstract: sparse entries exact), at full
-// occupancy.  No global atomics: the result is deterministic.  Waits are bounded.
+// positions arrive by bulk asynchronous copies while it stages the rest.  Each
+// lane then takes one word (EPW entries of one position) at a time: x'[s] is a
+// broadcast load, each centroid is one conflict-free 16-byte load, and each
+// product is added to its row with a shared-memory atomic.  The block writes its
+// row sums to its own fp32 plane of the caller's workspace, and k_cs_finalize
+// sums the planes per row, applies the row scale and adds the fused sparse
+// correction and the outlier-column block (SCVQ summary step 4; HAS-VQ abstract:
+// sparse entries exact), at full occupancy.  No global atomics.  Waits are
+// bounded.
 #include "vqlin_internal.cuh"
 
 namespace vqlin {
@@ -59,15 +60,14 @@ __host__ __device__ inline size_t r16(size_t v) { return (v + 15) & ~size_t(15);
 
 // Shared-memory layout of a block (byte offsets, every region 16-byte aligned).
 struct Carve {
-  size_t xs, yp, off, bar, words;
+  size_t xs, yp, bar, words;
   __host__ __device__ Carve(int E, int n_sub, int NB, int rpp) {
-    xs = r16((size_t)E * COPIES * 16);
+    xs = r16((size_t)(E + 1) * COPIES * 16);            // slice + the null entry
     yp = r16(xs + (size_t)n_sub * NB * 8 * 4);
-    off = r16(yp + (size_t)NB * rpp * 4);
-    bar = r16(off + (size_t)(n_sub + 1) * 4);
+    bar = r16(yp + (size_t)NB * rpp * 4);
     words = bar + 16;
   }
-  // entry words then their start positions (u16), for a buffer of `cap` words (cap % 8 == 0)
+  // entry words then their positions (u16), for a buffer of `cap` words (cap % 8 == 0)
   __host__ __device__ size_t wpos(int cap) const { return words + (size_t)cap * 8; }
   __host__ __device__ size_t total(int cap) const { return wpos(cap) + (size_t)cap * 2; }
 };
@@ -98,16 +98,15 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_cs(Args a) {
   uint4* cbs = reinterpret_cast<uint4*>(smem);                        // [E][8]
   float* xs = reinterpret_cast<float*>(smem + cv.xs);                 // [n_sub][NB][8]
   float* yp = reinterpret_cast<float*>(smem + cv.yp);                 // [NB][RPP]
-  int* off = reinterpret_cast<int*>(smem + cv.off);                   // [n_sub + 1]
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + cv.bar);         // mbarrier + abort flag
   uint64_t* words = reinterpret_cast<uint64_t*>(smem + cv.words);     // [cap]
   uint16_t* wpos = reinterpret_cast<uint16_t*>(smem + cv.wpos(a.words_cap));   // [cap]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // this block's words: entries [cs_start[c], cs_start[c+1]), a multiple of 8 words
-  const int64_t w_begin = L.cs_start[c] / EPW;
-  const int n_words = (int)((L.cs_start[c + 1] - L.cs_start[c]) / EPW);
+  // this block's words [cs_start[c], cs_start[c+1]), a multiple of 8
+  const int64_t w_begin = L.cs_start[c];
+  const int n_words = (int)(L.cs_start[c + 1] - w_begin);
   const bool one_chunk = n_words <= a.words_cap;
   auto issue_chunk = [&](int w0) {      // thread 0: words [w0, w0 + n) and their positions
     const int n = min(a.words_cap, n_words - w0);
@@ -124,16 +123,14 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_cs(Args a) {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     if (one_chunk && n_words > 0) issue_chunk(0);   // overlaps the staging below
   }
-  // ---- codebook slice (8 interleaved copies), x' per position, run counts; every
-  //      global load of this phase is issued before any of its values is used
+  // ---- codebook slice (8 interleaved copies), x' per position; every global load
+  //      of this phase is issued before any of its values is used
   {
     const uint4* cb = reinterpret_cast<const uint4*>(L.cb1) + slice0;
     uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
     const int k0 = threadIdx.x, k1 = threadIdx.x + THREADS;
     if (k0 < E_p) v0 = __ldg(cb + k0);
     if (k1 < E_p) v1 = __ldg(cb + k1);
-    const uint16_t* cnt = L.cs_counts + (size_t)c * n_sub;
-    int cnt0 = threadIdx.x < n_sub ? cnt[threadIdx.x] : 0;
     // x' for (position s, batch b), one item per thread per round: 16-byte loads of x and c when
     // the main columns are contiguous and 8-aligned, else eight clamped scalar loads
     const bool vec = !L.colmap && a.xt != VQLIN_F32 && (L.n_in & 7) == 0;
@@ -171,41 +168,32 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_cs(Args a) {
 #pragma unroll
           for (int k = 0; k < 8; ++k) if (!ok[k]) v[k] = 0.f;
         }
+        // item i fills 32 bytes; lanes 4..7 of each quarter-warp write their two halves in the
+        // other order, so every store instruction covers eight different bank groups
         float4* dst = reinterpret_cast<float4*>(xs + ((size_t)s * NB + b) * 8);
-        dst[0] = make_float4(v[0] * cvv[0], v[1] * cvv[1], v[2] * cvv[2], v[3] * cvv[3]);
-        dst[1] = make_float4(v[4] * cvv[4], v[5] * cvv[5], v[6] * cvv[6], v[7] * cvv[7]);
+        float4 lo = make_float4(v[0] * cvv[0], v[1] * cvv[1], v[2] * cvv[2], v[3] * cvv[3]);
+        float4 hi = make_float4(v[4] * cvv[4], v[5] * cvv[5], v[6] * cvv[6], v[7] * cvv[7]);
+        const int sw = (threadIdx.x >> 2) & 1;
+        dst[sw] = sw ? hi : lo;
+        dst[sw ^ 1] = sw ? lo : hi;
       }
     });
-    if (threadIdx.x < n_sub) off[threadIdx.x] = cnt0;
-    for (int s2 = threadIdx.x + THREADS; s2 < n_sub; s2 += THREADS) off[s2] = cnt[s2];
+    // the copies are written in a lane-rotated order: at every store the eight lanes of a
+    // quarter-warp write eight different copies, i.e. eight different bank groups
+    const int rot = threadIdx.x & (COPIES - 1);
     if (k0 < E_p)
 #pragma unroll
-      for (int cc = 0; cc < COPIES; ++cc) cbs[k0 * COPIES + cc] = v0;
+      for (int cc = 0; cc < COPIES; ++cc) cbs[k0 * COPIES + ((cc + rot) & (COPIES - 1))] = v0;
     if (k1 < E_p)
 #pragma unroll
-      for (int cc = 0; cc < COPIES; ++cc) cbs[k1 * COPIES + cc] = v1;
+      for (int cc = 0; cc < COPIES; ++cc) cbs[k1 * COPIES + ((cc + rot) & (COPIES - 1))] = v1;
     for (int k = threadIdx.x + 2 * THREADS; k < E_p; k += THREADS) {   // slices wider than 2*THREADS
       const uint4 v = __ldg(cb + k);
 #pragma unroll
-      for (int cc = 0; cc < COPIES; ++cc) cbs[k * COPIES + cc] = v;
+      for (int cc = 0; cc < COPIES; ++cc) cbs[k * COPIES + ((cc + rot) & (COPIES - 1))] = v;
     }
+    if (threadIdx.x < COPIES) cbs[E * COPIES + threadIdx.x] = make_uint4(0, 0, 0, 0);   // the null entry
     for (int i = threadIdx.x; i < NB * RPP; i += THREADS) yp[i] = 0.f;
-  }
-  __syncthreads();
-  if (warp == 0) {   // exclusive prefix sum of the counts
-    const int per = (n_sub + 31) / 32;
-    const int s0 = lane * per, s1 = min(n_sub, s0 + per);
-    int local = 0;
-    for (int s = s0; s < s1; ++s) local += off[s];
-    int incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    int run = incl - local;
-    for (int s = s0; s < s1; ++s) { const int cs = off[s]; off[s] = run; run += cs; }
-    if (lane == 31) off[n_sub] = incl;
   }
   __syncthreads();
 
@@ -213,7 +201,6 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_cs(Args a) {
   const uint32_t lmask = (1u << L.cs_local_bits) - 1u;
   const uint64_t emask = (1ull << L.cs_ebits) - 1ull;
   const int lbits = L.cs_local_bits;
-  const int n_ent = off[n_sub];                      // real entries (padding is never processed)
   uint32_t phase = 0;
   for (int w0 = 0; w0 < n_words; w0 += a.words_cap) {
     if (!one_chunk) {
@@ -233,13 +220,9 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_cs(Args a) {
     if (*abort_flag) break;
     const int nw = min(a.words_cap, n_words - w0);
     const int wb = nw * warp / WARPS, we = nw * (warp + 1) / WARPS;
-    float xr[NB][8];
-    int cur = -1;
     for (int wi = wb + lane; wi < we; wi += 32) {
-      const int e0 = (w0 + wi) * EPW;                // block-local index of the word's first entry
-      if (e0 >= n_ent) continue;
       const uint64_t wv = words[wi];
-      int s = wpos[wi];
+      const int s = wpos[wi];
       uint32_t ent[EPW];
       uint4 cen[EPW];
 #pragma unroll
@@ -247,29 +230,25 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_cs(Args a) {
         ent[u] = (uint32_t)((wv >> (u * SLOT)) & emask);
         cen[u] = cbs[(ent[u] & lmask) * COPIES + (lane & (COPIES - 1))];
       }
+      float xr[NB][8];
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        const float4* xv = reinterpret_cast<const float4*>(xs + ((size_t)s * NB + b) * 8);
+        const float4 x0 = xv[0], x1 = xv[1];
+        xr[b][0] = x0.x; xr[b][1] = x0.y; xr[b][2] = x0.z; xr[b][3] = x0.w;
+        xr[b][4] = x1.x; xr[b][5] = x1.y; xr[b][6] = x1.z; xr[b][7] = x1.w;
+      }
 #pragma unroll
       for (int u = 0; u < EPW; ++u) {
-        const int e = e0 + u;
-        if (e >= n_ent) break;
-        if (u > 0) while (off[s + 1] <= e) ++s;
-        if (s != cur) {
-          cur = s;
-#pragma unroll
-          for (int b = 0; b < NB; ++b) {
-            const float4* xv = reinterpret_cast<const float4*>(xs + ((size_t)s * NB + b) * 8);
-            const float4 x0 = xv[0], x1 = xv[1];
-            xr[b][0] = x0.x; xr[b][1] = x0.y; xr[b][2] = x0.z; xr[b][3] = x0.w;
-            xr[b][4] = x1.x; xr[b][5] = x1.y; xr[b][6] = x1.z; xr[b][7] = x1.w;
-          }
-        }
         const __half2* h2 = reinterpret_cast<const __half2*>(&cen[u]);
         float cf[8];
 #pragma unroll
         for (int k = 0; k < 4; ++k) { const float2 f2 = __half22float2(h2[k]); cf[2 * k] = f2.x; cf[2 * k + 1] = f2.y; }
         const int row_l = (int)(ent[u] >> lbits);
+        const bool real = (ent[u] & lmask) != (uint32_t)E;   // null entries add nothing
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
-          if (b >= B) continue;
+          if (b >= B || !real) continue;
           float p0 = cf[0] * xr[b][0], p1 = cf[1] * xr[b][1];
           p0 = fmaf(cf[2], xr[b][2], p0); p1 = fmaf(cf[3], xr[b][3], p1);
           p0 = fmaf(cf[4], xr[b][4], p0); p1 = fmaf(cf[5], xr[b][5], p1);
@@ -434,6 +413,7 @@ static cudaError_t launch_cfg(const Args& a, size_t smem, cudaStream_t s) {
   auto k = k_gemv_cs<NB, EPW>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  note_launches(1);
   k<<<a.L.cs_P * a.L.cs_H, THREADS, smem, s>>>(a);
   return cudaGetLastError();
 }
@@ -493,6 +473,7 @@ cudaError_t launch_gemv_cs(const Layer& L, const void* x, vqlin_dtype xt, int ba
   cfg.numAttrs = 1;
   const float* planes = a.planes;
   const int P = L.cs_P;
+  note_launches(1);
   if (NB == 1) e = cudaLaunchKernelEx(&cfg, k_cs_finalize<1>, L, planes, P, x, xt, batch, y, yt);
   else if (NB == 2) e = cudaLaunchKernelEx(&cfg, k_cs_finalize<2>, L, planes, P, x, xt, batch, y, yt);
   else e = cudaLaunchKernelEx(&cfg, k_cs_finalize<4>, L, planes, P, x, xt, batch, y, yt);

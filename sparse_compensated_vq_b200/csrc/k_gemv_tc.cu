@@ -634,6 +634,7 @@ static cudaError_t launch_wt_cfg(const Args& args, size_t smem, int grid, cudaSt
   auto k = k_gemv_wt<NT, W, CB_SMEM, COPIES>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  note_launches(1);
   k<<<grid, THREADS, smem, s>>>(args);
   return cudaGetLastError();
 }
@@ -670,6 +671,7 @@ static cudaError_t launch_cfg(const Args& args, size_t smem, int grid, cudaStrea
   auto k = k_gemv_tc<NT, W, CB_SMEM, COPIES>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  note_launches(1);
   k<<<grid, THREADS, smem, s>>>(args);
   return cudaGetLastError();
 }
@@ -782,6 +784,7 @@ cudaError_t launch_gemv_tc(const Layer& L, const void* x, vqlin_dtype xt, int ba
       if (e != cudaSuccess) return e;
       if (yt != VQLIN_F32) {
         int64_t n = (int64_t)batch * L.n_out;
+        note_launches(1);
         k_finalize<<<(int)((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024), 256, 0, s>>>(acc, n, y, yt);
         e = cudaGetLastError();
       }
@@ -812,6 +815,7 @@ cudaError_t launch_gemv_tc(const Layer& L, const void* x, vqlin_dtype xt, int ba
   if (e != cudaSuccess) return e;
   if (a.split && yt != VQLIN_F32) {
     int64_t n = (int64_t)batch * L.n_out;
+    note_launches(1);
     k_finalize<<<(int)((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024), 256, 0, s>>>(a.acc, n, y, yt);
     e = cudaGetLastError();
   }

@@ -41,21 +41,24 @@ struct Layer {
   int32_t n_ls;                         // layout slabs per row
   int64_t tstride;                      // bytes per row = n_ls * 8 * w
   // Codebook-stationary layout (large single-stage codebooks, d = 8; null otherwise):
-  // block c = p * cs_H + h owns codebook slice p (entries [p*cs_E, (p+1)*cs_E)) and row half h
-  // (rows [h*cs_rpp, ...)); its entries (row - h*cs_rpp) << cs_local_bits | (index - p*cs_E),
-  // cs_ebits wide, cs_epw per 64-bit word in slots of 21 (cs_epw = 3) or 32 bits (cs_epw = 2),
-  // sorted by position then row, start at entry
-  // cs_start[c] (a multiple of 8*cs_epw); cs_counts[c*n_sub + s] entries at position s.
+  // block c = p * cs_H + h owns codebook slice p (entries [p*cs_E, (p+1)*cs_E), cs_E < 1024)
+  // and row half h (rows [h*cs_rpp, ...)); its entries (row - h*cs_rpp) << cs_local_bits |
+  // (index - p*cs_E), cs_ebits wide, cs_epw per 64-bit word in slots of 21 (cs_epw = 3) or 32
+  // bits (cs_epw = 2), sorted by position then row.  Every run of one position is padded to
+  // whole words with the null entry (row 0, local index cs_E: a zero centroid), so all
+  // entries of a word share the position cs_wpos[word]; block c's words are
+  // [cs_start[c], cs_start[c+1]) (multiples of 8, padded with null words).
   const uint64_t* cs_words;
-  const int64_t* cs_start;              // [cs_P*cs_H + 1]
-  const uint16_t* cs_counts;            // [cs_P*cs_H][n_sub]
-  const uint16_t* cs_wpos;              // position of the first entry of every word
+  const int64_t* cs_start;              // [cs_P*cs_H + 1], in words
+  const uint16_t* cs_wpos;              // position of every word
   int32_t cs_P, cs_H, cs_E, cs_rpp, cs_local_bits, cs_ebits, cs_epw;
   int64_t cs_max_words;                 // largest block's word count
 };
 
 // Last-error plumbing (thread-local detail string).
 void set_error(const char* fmt, ...);
+// Counts every kernel the library enqueues (exported as vqlin_kernel_launches).
+void note_launches(int n);
 vqlin_status cuda_status(cudaError_t e, const char* what);
 
 // Kernel launchers (return cudaGetLastError() of the launch).

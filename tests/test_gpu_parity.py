@@ -407,3 +407,22 @@ def test_gemv_codebook_stationary_full_qproj(vq):
         y = m.gemv_ws(x, out_dtype=torch.float16)
         torch.cuda.synchronize()
         G.assert_close(G.to_f64(y), oracle.gemv_f64(L, synth.bits_to_f64(xb[:batch], "f16")), "f16", "qproj cs B=%d" % batch)
+
+
+def test_kernel_launch_counter(vq):
+    """Every call enqueues at least one of the library's kernels and the counter sees each one."""
+    import torch
+    L, xb = G.workload("qproj")
+    m = vq.VQLinear(L)
+    x = G.torch_x(xb[:1], "f16")
+    n0 = vq.vqlin_kernel_launches()
+    m.gemv_ws(x, out_dtype=torch.float16)
+    n1 = vq.vqlin_kernel_launches()
+    assert n1 - n0 == 2          # codebook-stationary slice kernel + finalize
+    s = SMALL[0]
+    ms = vq.VQLinear(s)
+    n0 = vq.vqlin_kernel_launches()
+    ms.gemv(G.torch_x(synth.activations(np.random.default_rng(1), 2, s.n_in, "f16"), "f16"))
+    ms.dequant()
+    torch.cuda.synchronize()
+    assert vq.vqlin_kernel_launches() - n0 >= 2
