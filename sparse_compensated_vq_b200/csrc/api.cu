@@ -337,28 +337,29 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
   std::vector<uint64_t> cs_words;
   std::vector<int64_t> cs_start;
   std::vector<uint16_t> cs_wpos;
+  std::vector<float> cs_bound;
   int32_t cs_P = 0, cs_H = 0, cs_E = 0, cs_rpp = 0, cs_lbits = 0, cs_ebits = 0, cs_epw = 0;
   if (d == 8 && D->k2 == 0 && D->k1 > 10240 && n_sub > 0 && n_sub <= 65536) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     auto bitlen = [](int64_t v) { int b = 0; while ((1ll << b) <= v) ++b; return b < 1 ? 1 : b; };
-    int H = D->n_out >= 2048 ? 2 : 1;
+    const int H = D->n_out >= 2048 ? 2 : 1;
     int P = (int)std::max<int64_t>(ceil_div(D->k1, 1023), std::max(1, sms / H));
     P = std::min(P, D->k1);
-    int E = (int)ceil_div(D->k1, P);
+    const int E = (int)ceil_div(D->k1, P);
     P = (int)ceil_div(D->k1, E);
-    int rpp = (int)ceil_div(D->n_out, H);
-    int lb = bitlen(E), rb = bitlen(rpp - 1), eb = lb + rb;     // local indices 0..E (E = null entry)
-    int epw = eb <= 21 ? 3 : (eb <= 32 ? 2 : 0);
+    const int rpp = (int)ceil_div(D->n_out, H);
+    const int lb = bitlen(E), rb = bitlen(rpp - 1), eb = lb + rb;   // local indices 0..E (E = null entry)
+    const int epw = eb <= 21 ? 3 : (eb <= 32 ? 2 : 0);
     if (epw && rpp <= 65535) {
-      cs_P = P; cs_H = H; cs_E = E; cs_rpp = rpp; cs_lbits = lb; cs_ebits = eb; cs_epw = epw;
       const int ncta = P * H;
       const int slot = epw == 3 ? 21 : 32;
       const uint32_t null_entry = (uint32_t)E;                  // row 0, zero centroid
       std::vector<std::vector<uint64_t>> bw(ncta);              // words of every block
       std::vector<std::vector<uint16_t>> bp(ncta);              // their positions
       std::vector<int> fill(ncta, 0);                           // entries in the block's open word
+      std::vector<int32_t> per_row((size_t)ncta * rpp, 0);      // entries of every (block, row)
       auto put = [&](int cc, uint32_t ent, int32_t sv) {
         if (fill[cc] == 0) { bw[cc].push_back(0); bp[cc].push_back((uint16_t)sv); }
         bw[cc].back() |= (uint64_t)ent << (fill[cc] * slot);
@@ -367,21 +368,46 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
       for (int32_t sv = 0; sv < n_sub; ++sv) {
         for (int32_t i = 0; i < D->n_out; ++i) {
           uint32_t idx = host_field(codes.data() + (size_t)i * D->row_stride_bytes, sv, w) & m1;
-          int pp = (int)(idx / (uint32_t)E), hh = i / rpp;
-          put(pp * H + hh, ((uint32_t)(i - hh * rpp) << lb) | (idx - (uint32_t)pp * E), sv);
+          const int pp = (int)(idx / (uint32_t)E), hh = i / rpp, cc = pp * H + hh;
+          put(cc, ((uint32_t)(i - hh * rpp) << lb) | (idx - (uint32_t)pp * E), sv);
+          per_row[(size_t)cc * rpp + (i - hh * rpp)] += 1;
         }
         for (int cc = 0; cc < ncta; ++cc)   // close the run of position sv
           while (fill[cc] != 0) put(cc, null_entry, sv);
       }
-      uint64_t null_word = 0;
-      for (int u = 0; u < epw; ++u) null_word |= (uint64_t)null_entry << (u * slot);
-      cs_start.assign(ncta + 1, 0);
-      for (int cc = 0; cc < ncta; ++cc) cs_start[cc + 1] = cs_start[cc] + round_up((int64_t)bw[cc].size(), 8);
-      cs_words.assign((size_t)cs_start[ncta], null_word);
-      cs_wpos.assign(cs_words.size(), 0);
+      // Fixed-point bound of every block: (most entries of one row in the block) * (largest l1
+      // norm of a centroid of its slice).  Every product satisfies |c . x'| <= l1(c) * max|x'|,
+      // so a row's partial sum in the block stays below bound * max|x'|.
+      const uint16_t* C1 = as<uint16_t>(cb1);
+      std::vector<double> l1(P, 0.0);
+      for (int32_t k = 0; k < D->k1; ++k) {
+        double a1 = 0;
+        for (int t = 0; t < 8; ++t) a1 += std::fabs(f16_val(C1[(size_t)k * 8 + t]));
+        l1[k / E] = std::max(l1[k / E], a1);
+      }
+      std::vector<float> bound(ncta, 0.f);
+      int64_t max_cnt = 0;
       for (int cc = 0; cc < ncta; ++cc) {
-        std::copy(bw[cc].begin(), bw[cc].end(), cs_words.begin() + cs_start[cc]);
-        std::copy(bp[cc].begin(), bp[cc].end(), cs_wpos.begin() + cs_start[cc]);
+        int32_t m = 0;
+        for (int r = 0; r < rpp; ++r) m = std::max(m, per_row[(size_t)cc * rpp + r]);
+        max_cnt = std::max<int64_t>(max_cnt, m);
+        bound[cc] = std::nextafter((float)((double)m * l1[cc / H]), INFINITY);
+      }
+      // A row's fixed-point rounding error is at most n_sub * max_cnt * 2^-31 times the
+      // largest possible single product (k_gemv_cs.cu); past 2^20 the layout is not used.
+      if ((int64_t)n_sub * max_cnt <= (1ll << 20)) {
+        cs_P = P; cs_H = H; cs_E = E; cs_rpp = rpp; cs_lbits = lb; cs_ebits = eb; cs_epw = epw;
+        uint64_t null_word = 0;
+        for (int u = 0; u < epw; ++u) null_word |= (uint64_t)null_entry << (u * slot);
+        cs_start.assign(ncta + 1, 0);
+        for (int cc = 0; cc < ncta; ++cc) cs_start[cc + 1] = cs_start[cc] + round_up((int64_t)bw[cc].size(), 8);
+        cs_words.assign((size_t)cs_start[ncta], null_word);
+        cs_wpos.assign(cs_words.size(), 0);
+        for (int cc = 0; cc < ncta; ++cc) {
+          std::copy(bw[cc].begin(), bw[cc].end(), cs_words.begin() + cs_start[cc]);
+          std::copy(bp[cc].begin(), bp[cc].end(), cs_wpos.begin() + cs_start[cc]);
+        }
+        cs_bound = std::move(bound);
       }
     }
   }
@@ -418,6 +444,7 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
     L.cs_words = up.put<uint64_t>(cs_words.data(), cs_words.size() * 8);
     L.cs_start = up.put<int64_t>(cs_start.data(), cs_start.size() * 8);
     L.cs_wpos = up.put<uint16_t>(cs_wpos.data(), cs_wpos.size() * 2);
+    L.cs_bound = up.put<float>(cs_bound.data(), cs_bound.size() * 4);
     L.cs_P = cs_P; L.cs_H = cs_H; L.cs_E = cs_E; L.cs_rpp = cs_rpp;
     L.cs_local_bits = cs_lbits; L.cs_ebits = cs_ebits; L.cs_epw = cs_epw;
     L.cs_max_words = 0;

@@ -51,6 +51,7 @@ struct Layer {
   const uint64_t* cs_words;
   const int64_t* cs_start;              // [cs_P*cs_H + 1], in words
   const uint16_t* cs_wpos;              // position of every word
+  const float* cs_bound;                // [cs_P*cs_H]: (most entries of one row) * max l1(centroid)
   int32_t cs_P, cs_H, cs_E, cs_rpp, cs_local_bits, cs_ebits, cs_epw;
   int64_t cs_max_words;                 // largest block's word count
 };

@@ -426,3 +426,13 @@ def test_kernel_launch_counter(vq):
     ms.dequant()
     torch.cuda.synchronize()
     assert vq.vqlin_kernel_launches() - n0 >= 2
+
+
+def test_codebook_stationary_is_deterministic(vq):
+    """The fixed-point row sums do not depend on the order of the atomics: repeated calls agree bit for bit."""
+    import torch
+    L, xb = G.workload("qproj")
+    m = vq.VQLinear(L)
+    x = G.torch_x(xb[:4], "f16")
+    ys = [m.gemv_ws(x, out_dtype=torch.float32).cpu().numpy().view(np.uint32) for _ in range(3)]
+    assert (ys[0] == ys[1]).all() and (ys[0] == ys[2]).all()
