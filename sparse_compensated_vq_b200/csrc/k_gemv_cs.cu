@@ -128,8 +128,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_cs(Args a) {
     bulk_load(words, L.cs_words + w_begin + w0, (uint32_t)(n * 8), su32(bar));
     bulk_load(wpos, L.cs_wpos + w_begin + w0, (uint32_t)(n * 2), su32(bar));
   };
-  // the finalize kernel may start now: its sparse/outlier work does not read this grid's output
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // Launched as a programmatic dependent: everything before griddepcontrol.wait reads only
+  // the layer (immutable) and writes only shared memory, so it may overlap the previous grid.
   if (threadIdx.x == 0) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(su32(bar)) : "memory");
     *abort_flag = 0;
@@ -137,8 +137,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_cs(Args a) {
     if (one_chunk && n_words > 0) issue_chunk(0);   // overlaps the staging below
   }
   float fx_scale, fx_inv;                            // fixed-point scale S and 1/S
-  // ---- codebook slice (8 interleaved copies), x' per position; every global load
-  //      of this phase is issued before any of its values is used
+  // ---- codebook slice (8 interleaved copies), then x' per position
   {
     const float bound = L.cs_bound[c];
     float xmax = 0.f;
@@ -147,6 +146,27 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_cs(Args a) {
     const int k0 = threadIdx.x, k1 = threadIdx.x + THREADS;
     if (k0 < E_p) v0 = __ldg(cb + k0);
     if (k1 < E_p) v1 = __ldg(cb + k1);
+    // the copies are written in a lane-rotated order: at every store the eight lanes of a
+    // quarter-warp write eight different copies, i.e. eight different bank groups
+    const int rot = threadIdx.x & (COPIES - 1);
+    if (k0 < E_p)
+#pragma unroll
+      for (int cc = 0; cc < COPIES; ++cc) cbs[k0 * COPIES + ((cc + rot) & (COPIES - 1))] = v0;
+    if (k1 < E_p)
+#pragma unroll
+      for (int cc = 0; cc < COPIES; ++cc) cbs[k1 * COPIES + ((cc + rot) & (COPIES - 1))] = v1;
+    for (int k = threadIdx.x + 2 * THREADS; k < E_p; k += THREADS) {   // slices wider than 2*THREADS
+      const uint4 v = __ldg(cb + k);
+#pragma unroll
+      for (int cc = 0; cc < COPIES; ++cc) cbs[k * COPIES + ((cc + rot) & (COPIES - 1))] = v;
+    }
+    if (threadIdx.x < COPIES) cbs[E * COPIES + threadIdx.x] = make_uint4(0, 0, 0, 0);   // the null entry
+    for (int i = threadIdx.x; i < NB * RPP; i += THREADS) yp[i] = 0;
+
+    // x is written by the previous grid: wait for it.  Only then may the finalize grid start
+    // (its sparse and outlier terms read x before they wait for this grid).
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     // x' for (position s, batch b), one item per thread per round: 16-byte loads of x and c when
     // the main columns are contiguous and 8-aligned, else eight clamped scalar loads
     const bool vec = !L.colmap && a.xt != VQLIN_F32 && (L.n_in & 7) == 0;
@@ -196,22 +216,6 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_cs(Args a) {
         dst[sw ^ 1] = sw ? lo : hi;
       }
     });
-    // the copies are written in a lane-rotated order: at every store the eight lanes of a
-    // quarter-warp write eight different copies, i.e. eight different bank groups
-    const int rot = threadIdx.x & (COPIES - 1);
-    if (k0 < E_p)
-#pragma unroll
-      for (int cc = 0; cc < COPIES; ++cc) cbs[k0 * COPIES + ((cc + rot) & (COPIES - 1))] = v0;
-    if (k1 < E_p)
-#pragma unroll
-      for (int cc = 0; cc < COPIES; ++cc) cbs[k1 * COPIES + ((cc + rot) & (COPIES - 1))] = v1;
-    for (int k = threadIdx.x + 2 * THREADS; k < E_p; k += THREADS) {   // slices wider than 2*THREADS
-      const uint4 v = __ldg(cb + k);
-#pragma unroll
-      for (int cc = 0; cc < COPIES; ++cc) cbs[k * COPIES + ((cc + rot) & (COPIES - 1))] = v;
-    }
-    if (threadIdx.x < COPIES) cbs[E * COPIES + threadIdx.x] = make_uint4(0, 0, 0, 0);   // the null entry
-    for (int i = threadIdx.x; i < NB * RPP; i += THREADS) yp[i] = 0;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) xmax = fmaxf(xmax, __shfl_xor_sync(0xffffffffu, xmax, o));
     if (lane == 0) wmax[warp] = xmax;
@@ -319,6 +323,8 @@ __global__ void __launch_bounds__(256) k_cs_finalize(Layer L, const float* __res
   __shared__ float part[8][NB][32], spv[NB][32], ovv[NB][32];
   const int i0 = blockIdx.x * 32;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  // the next grid may start its layer-only prologue; it waits for this grid before reading x
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   with_dtype(xt, [&](auto tag) {
     constexpr int XT = decltype(tag)::value;
     // sparse term of rows i0 + 4*warp .. +3
@@ -439,14 +445,29 @@ __global__ void __launch_bounds__(256) k_cs_finalize(Layer L, const float* __res
   }
 }
 
+// Both grids are launched as programmatic dependents of whatever precedes them on the stream.
+static cudaLaunchConfig_t pdl_config(dim3 grid, int threads, size_t smem, cudaStream_t s, cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg = {};
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
 template <int NB, int EPW>
 static cudaError_t launch_cfg(const Args& a, size_t smem, cudaStream_t s) {
   auto k = k_gemv_cs<NB, EPW>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[1];
+  const cudaLaunchConfig_t cfg = pdl_config(dim3(a.L.cs_P * a.L.cs_H), THREADS, smem, s, attr);
   note_launches(1);
-  k<<<a.L.cs_P * a.L.cs_H, THREADS, smem, s>>>(a);
-  return cudaGetLastError();
+  return cudaLaunchKernelEx(&cfg, k, a);
 }
 
 }  // namespace csg
@@ -492,16 +513,8 @@ cudaError_t launch_gemv_cs(const Layer& L, const void* x, vqlin_dtype xt, int ba
     else e = launch_cfg<4, 2>(a, smem, s);
   }
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.gridDim = dim3((L.n_out + 31) / 32);
-  cfg.blockDim = dim3(256);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = s;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  const cudaLaunchConfig_t cfg = pdl_config(dim3((L.n_out + 31) / 32), 256, 0, s, attr);
   const float* planes = a.planes;
   const int P = L.cs_P;
   note_launches(1);
