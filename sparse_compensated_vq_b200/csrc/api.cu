@@ -399,8 +399,52 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
         cs_P = P; cs_H = H; cs_E = E; cs_rpp = rpp; cs_lbits = lb; cs_ebits = eb; cs_epw = epw;
         uint64_t null_word = 0;
         for (int u = 0; u < epw; ++u) null_word |= (uint64_t)null_entry << (u * slot);
+        const uint64_t emask = (1ull << eb) - 1ull;
         cs_start.assign(ncta + 1, 0);
-        for (int cc = 0; cc < ncta; ++cc) cs_start[cc + 1] = cs_start[cc] + round_up((int64_t)bw[cc].size(), 8);
+        for (int cc = 0; cc < ncta; ++cc) {
+          // whole groups of 32 words (one warp instruction covers one group)
+          while (bw[cc].size() % 32) { bw[cc].push_back(null_word); bp[cc].push_back(0); }
+          cs_start[cc + 1] = cs_start[cc] + (int64_t)bw[cc].size();
+          // Inside a group, deal the entries of every position run to the slots so that the
+          // rows that one slot column sends to the shared-memory accumulator fall in different
+          // banks (row mod 32): greedy, each entry to the open slot whose column holds the
+          // fewest rows of its bank so far.
+          for (size_t g0 = 0; g0 < bw[cc].size(); g0 += 32) {
+            int cnt[3][32] = {};
+            size_t w = g0;
+            while (w < g0 + 32) {
+              size_t w1 = w + 1;
+              while (w1 < g0 + 32 && bp[cc][w1] == bp[cc][w]) ++w1;
+              const int m = (int)(w1 - w);
+              std::vector<uint32_t> ents;
+              for (size_t q = w; q < w1; ++q)
+                for (int u = 0; u < epw; ++u) {
+                  const uint32_t e = (uint32_t)((bw[cc][q] >> (u * slot)) & emask);
+                  if ((e & ((1u << lb) - 1u)) != null_entry) ents.push_back(e);
+                }
+              std::vector<std::vector<uint32_t>> col(epw);
+              for (uint32_t e : ents) {
+                const int bank = (int)((e >> lb) & 31u);
+                int best = -1;
+                for (int u = 0; u < epw; ++u) {
+                  if ((int)col[u].size() >= m) continue;
+                  if (best < 0 || cnt[u][bank] < cnt[best][bank] ||
+                      (cnt[u][bank] == cnt[best][bank] && col[u].size() < col[best].size()))
+                    best = u;
+                }
+                col[best].push_back(e);
+                cnt[best][bank] += 1;
+              }
+              for (int j = 0; j < m; ++j) {
+                uint64_t word = 0;
+                for (int u = 0; u < epw; ++u)
+                  word |= (uint64_t)(j < (int)col[u].size() ? col[u][j] : null_entry) << (u * slot);
+                bw[cc][w + j] = word;
+              }
+              w = w1;
+            }
+          }
+        }
         cs_words.assign((size_t)cs_start[ncta], null_word);
         cs_wpos.assign(cs_words.size(), 0);
         for (int cc = 0; cc < ncta; ++cc) {

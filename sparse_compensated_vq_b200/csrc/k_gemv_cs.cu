@@ -79,7 +79,7 @@ struct Carve {
     bar = r16(yp + (size_t)NB * rpp * 4);
     words = bar + 16 + WARPS * 4;                     // mbarrier, abort flag, per-warp max|x'|
   }
-  // entry words then their positions (u16), for a buffer of `cap` words (cap % 8 == 0)
+  // entry words then their positions (u16), for a buffer of `cap` words (cap % 32 == 0)
   __host__ __device__ size_t wpos(int cap) const { return words + (size_t)cap * 8; }
   __host__ __device__ size_t total(int cap) const { return wpos(cap) + (size_t)cap * 2; }
 };
@@ -90,7 +90,7 @@ struct Args {
   vqlin_dtype xt;
   int batch;
   float* planes;        // [P][batch][n_out]
-  int words_cap;        // words the shared buffer holds (a multiple of 8)
+  int words_cap;        // words the shared buffer holds (a multiple of 32)
 };
 
 template <int NB, int EPW>
@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_cs(Args a) {
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // this block's words [cs_start[c], cs_start[c+1]), a multiple of 8
+  // this block's words [cs_start[c], cs_start[c+1]), a multiple of 32
   const int64_t w_begin = L.cs_start[c];
   const int n_words = (int)(L.cs_start[c + 1] - w_begin);
   const bool one_chunk = n_words <= a.words_cap;
@@ -253,8 +253,9 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_cs(Args a) {
     }
     __syncthreads();
     if (*abort_flag) break;
-    const int nw = min(a.words_cap, n_words - w0);
-    const int wb = nw * warp / WARPS, we = nw * (warp + 1) / WARPS;
+    // warps take whole groups of 32 words, so one instruction covers one layout group
+    const int ng = min(a.words_cap, n_words - w0) >> 5;
+    const int wb = (ng * warp / WARPS) << 5, we = (ng * (warp + 1) / WARPS) << 5;
     for (int wi = wb + lane; wi < we; wi += 32) {
       const uint64_t wv = words[wi];
       const int s = wpos[wi];
@@ -407,6 +408,12 @@ __global__ void __launch_bounds__(256) k_cs_finalize(Layer L, const float* __res
       }
     }
   });
+  // row scale of this thread's output row (layer data, read before the wait)
+  float rsc = 1.f;
+  {
+    const int i = i0 + (t & 31);
+    if (L.rs && (t >> 5) < NB && i < L.n_out) rsc = __half2float(L.rs[i]);
+  }
   // the planes are written by the preceding codebook-stationary grid
   asm volatile("griddepcontrol.wait;" ::: "memory");
   {
@@ -439,7 +446,6 @@ __global__ void __launch_bounds__(256) k_cs_finalize(Layer L, const float* __res
       float body = 0.f;
 #pragma unroll
       for (int g = 0; g < 8; ++g) body += part[g][b][r];
-      const float rsc = L.rs ? __half2float(L.rs[i]) : 1.f;
       store_from_float(y, yt, (int64_t)b * L.n_out + i, fmaf(rsc, body + ovv[b][r], spv[b][r]));
     }
   }
@@ -497,10 +503,10 @@ cudaError_t launch_gemv_cs(const Layer& L, const void* x, vqlin_dtype xt, int ba
   if (cv.total(64) > smem_max) return cudaSuccess;
   Args a;
   a.L = L; a.x = x; a.xt = xt; a.batch = batch; a.planes = reinterpret_cast<float*>(ws);
-  int cap = (int)(((smem_max - cv.words) / 10) & ~7ll);      // 8 + 2 bytes per word, whole groups of 8
-  const int need_words = (int)((L.cs_max_words + 7) & ~7ll);
+  int cap = (int)(((smem_max - cv.words) / 10) & ~31ll);     // 8 + 2 bytes per word, whole groups of 32
+  const int need_words = (int)((L.cs_max_words + 31) & ~31ll);
   if (need_words < cap) cap = need_words;
-  a.words_cap = cap < 8 ? 8 : cap;
+  a.words_cap = cap < 32 ? 32 : cap;
   const size_t smem = cv.total(a.words_cap);
   cudaError_t e;
   if (L.cs_epw == 3) {

@@ -47,7 +47,9 @@ struct Layer {
   // bits (cs_epw = 2), sorted by position then row.  Every run of one position is padded to
   // whole words with the null entry (row 0, local index cs_E: a zero centroid), so all
   // entries of a word share the position cs_wpos[word]; block c's words are
-  // [cs_start[c], cs_start[c+1]) (multiples of 8, padded with null words).
+  // [cs_start[c], cs_start[c+1]) (multiples of 32, padded with null words).  Within each
+  // aligned group of 32 words the entries of a run are dealt to the slots so that a slot
+  // column's rows spread over the 32 banks.
   const uint64_t* cs_words;
   const int64_t* cs_start;              // [cs_P*cs_H + 1], in words
   const uint16_t* cs_wpos;              // position of every word
