@@ -144,8 +144,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_cs(Args a) {
     const uint4* cb = reinterpret_cast<const uint4*>(L.cb1) + slice0;
     uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
     const int k0 = threadIdx.x, k1 = threadIdx.x + THREADS;
-    if (k0 < E_p) v0 = __ldg(cb + k0);
-    if (k1 < E_p) v1 = __ldg(cb + k1);
+    v0 = __ldg(cb + min(k0, E_p - 1));                  // every slice holds at least one entry
+    v1 = __ldg(cb + min(k1, E_p - 1));
     // the copies are written in a lane-rotated order: at every store the eight lanes of a
     // quarter-warp write eight different copies, i.e. eight different bank groups
     const int rot = threadIdx.x & (COPIES - 1);
@@ -345,12 +345,13 @@ __global__ void __launch_bounds__(256) k_cs_finalize(Layer L, const float* __res
         float dl[8];
         int jj[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int e = e0 + 32 * u;
-          const bool ok = e < e_end;
-          dl[u] = ok ? L.delta[e] : 0.f;
-          jj[u] = ok ? (L.col16 ? (int)L.col16[e] : L.col[e]) : 0;
+        for (int u = 0; u < 8; ++u) {   // clamped indices: the eight loads issue together
+          const int e = min(e0 + 32 * u, e_end - 1);
+          dl[u] = L.delta[e];
+          jj[u] = L.col16 ? (int)L.col16[e] : L.col[e];
         }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) if (e0 + 32 * u >= e_end) dl[u] = 0.f;
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
           if (b >= batch) continue;
@@ -429,10 +430,10 @@ __global__ void __launch_bounds__(256) k_cs_finalize(Layer L, const float* __res
 #pragma unroll
           for (int k = 0; k < PG; ++k) {
             const int q = q0 + 8 * k;
-            v[k] = q < P ? pp[(size_t)q * stride] : 0.f;
+            v[k] = __ldcg(pp + (size_t)min(q, P - 1) * stride);   // clamped: every load issues at once
           }
 #pragma unroll
-          for (int k = 0; k < PG; ++k) acc += v[k];
+          for (int k = 0; k < PG; ++k) acc += (q0 + 8 * k < P) ? v[k] : 0.f;
         }
       }
       part[g][b][r] = acc;
