@@ -163,31 +163,58 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_cs(Args a) {
     if (threadIdx.x < COPIES) cbs[E * COPIES + threadIdx.x] = make_uint4(0, 0, 0, 0);   // the null entry
     for (int i = threadIdx.x; i < NB * RPP; i += THREADS) yp[i] = 0;
 
+    // column scales of every (position, batch) item, before the wait (layer data), parked in
+    // the item's x' slot; item i fills 32 bytes, and lanes 4..7 of each quarter-warp write
+    // their two halves in the other order, so every store covers eight different bank groups
+    const int sw = (threadIdx.x >> 2) & 1;
+    for (int i = threadIdx.x; i < n_sub * NB; i += THREADS) {
+      const int s = i / NB, b = i - s * NB;
+      const int q0 = s * 8;
+      float cvv[8];
+      if (!L.cs) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) cvv[k] = 1.f;
+      } else if (!L.colmap && q0 + 8 <= L.n_main) {
+        const uint4 cu = __ldg(reinterpret_cast<const uint4*>(L.cs + q0));
+        const __half* ch = reinterpret_cast<const __half*>(&cu);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) cvv[k] = __half2float(ch[k]);
+      } else {
+        int jj[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int q = min(q0 + k, L.n_main - 1);
+          jj[k] = L.colmap ? L.colmap[q] : q;
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) cvv[k] = __half2float(L.cs[jj[k]]);
+      }
+      float4* dst = reinterpret_cast<float4*>(xs + ((size_t)s * NB + b) * 8);
+      const float4 lo = make_float4(cvv[0], cvv[1], cvv[2], cvv[3]), hi = make_float4(cvv[4], cvv[5], cvv[6], cvv[7]);
+      dst[sw] = sw ? hi : lo;
+      dst[sw ^ 1] = sw ? lo : hi;
+    }
+
     // x is written by the previous grid: wait for it.  Only then may the finalize grid start
     // (its sparse and outlier terms read x before they wait for this grid).
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    // x' for (position s, batch b), one item per thread per round: 16-byte loads of x and c when
-    // the main columns are contiguous and 8-aligned, else eight clamped scalar loads
+    // x' = c (.) x for every item (the same thread owns the same items as above): 16-byte loads
+    // of x when the main columns are contiguous and 8-aligned, else eight clamped scalar loads
     const bool vec = !L.colmap && a.xt != VQLIN_F32 && (L.n_in & 7) == 0;
     with_dtype(a.xt, [&](auto tag) {
       constexpr int XT = decltype(tag)::value;
       for (int i = threadIdx.x; i < n_sub * NB; i += THREADS) {
         const int s = i / NB, b = i - s * NB;
         const int q0 = s * 8;
-        float v[8], cvv[8];
+        float v[8];
         if (XT != VQLIN_F32 && vec && b < B && q0 + 8 <= L.n_main) {
           const uint4 u = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const unsigned short*>(a.x) +
                                                               (int64_t)b * L.n_in + q0));
-          uint4 cu = make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);   // fp16 ones
-          if (L.cs) cu = __ldg(reinterpret_cast<const uint4*>(L.cs + q0));
           const unsigned short* hs = reinterpret_cast<const unsigned short*>(&u);
-          const __half* ch = reinterpret_cast<const __half*>(&cu);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
+          for (int k = 0; k < 8; ++k)
             v[k] = XT == VQLIN_F16 ? __half2float(__ushort_as_half(hs[k])) : __bfloat162float(__ushort_as_bfloat16(hs[k]));
-            cvv[k] = __half2float(ch[k]);
-          }
         } else {
           int jj[8];
           bool ok[8];
@@ -200,18 +227,14 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_cs(Args a) {
 #pragma unroll
           for (int k = 0; k < 8; ++k) v[k] = ldx<XT>(a.x, (int64_t)(b < B ? b : 0) * L.n_in + jj[k]);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) cvv[k] = L.cs ? __half2float(L.cs[jj[k]]) : 1.f;
-#pragma unroll
           for (int k = 0; k < 8; ++k) if (!ok[k]) v[k] = 0.f;
         }
-        // item i fills 32 bytes; lanes 4..7 of each quarter-warp write their two halves in the
-        // other order, so every store instruction covers eight different bank groups
         float4* dst = reinterpret_cast<float4*>(xs + ((size_t)s * NB + b) * 8);
-        float4 lo = make_float4(v[0] * cvv[0], v[1] * cvv[1], v[2] * cvv[2], v[3] * cvv[3]);
-        float4 hi = make_float4(v[4] * cvv[4], v[5] * cvv[5], v[6] * cvv[6], v[7] * cvv[7]);
+        const float4 c0 = dst[0], c1 = dst[1];
+        const float4 lo = make_float4(v[0] * c0.x, v[1] * c0.y, v[2] * c0.z, v[3] * c0.w);
+        const float4 hi = make_float4(v[4] * c1.x, v[5] * c1.y, v[6] * c1.z, v[7] * c1.w);
         xmax = fmaxf(xmax, fmaxf(fmaxf(fmaxf(fabsf(lo.x), fabsf(lo.y)), fmaxf(fabsf(lo.z), fabsf(lo.w))),
                                  fmaxf(fmaxf(fabsf(hi.x), fabsf(hi.y)), fmaxf(fabsf(hi.z), fabsf(hi.w)))));
-        const int sw = (threadIdx.x >> 2) & 1;
         dst[sw] = sw ? hi : lo;
         dst[sw ^ 1] = sw ? lo : hi;
       }
