@@ -85,6 +85,8 @@ __global__ void __launch_bounds__(kThreads) k_gemv_generic(Layer L, const void* 
     (void)n16;
     cb1 = cb1s; cb2 = L.cb2 ? cb2s : nullptr; cbo = cbos;
   }
+  pdl_wait();      // x and y belong to the previous grid until it completes
+  pdl_release();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row0 = blockIdx.x * kRowsPerCta + warp * kRPW;
   const uint32_t m1 = (1u << L.bits1) - 1u;
@@ -207,14 +209,12 @@ static cudaError_t launch_generic_nb(const Layer& L, const void* x, vqlin_dtype 
     auto k = k_gemv_generic<D, NB, true>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    note_launches(1);
-    k<<<grid, kThreads, smem, s>>>(L, x, xt, batch, y, yt, chunk);
+    return launch_pdl(k, dim3(grid), kThreads, smem, s, L, x, xt, batch, y, yt, chunk);
   } else {
     auto k = k_gemv_generic<D, NB, false>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    note_launches(1);
-    k<<<grid, kThreads, smem, s>>>(L, x, xt, batch, y, yt, chunk);
+    return launch_pdl(k, dim3(grid), kThreads, smem, s, L, x, xt, batch, y, yt, chunk);
   }
   return cudaGetLastError();
 }

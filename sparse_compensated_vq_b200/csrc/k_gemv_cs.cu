@@ -197,8 +197,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_cs(Args a) {
 
     // x is written by the previous grid: wait for it.  Only then may the finalize grid start
     // (its sparse and outlier terms read x before they wait for this grid).
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    pdl_wait();
+    pdl_release();
     // x' = c (.) x for every item (the same thread owns the same items as above): 16-byte loads
     // of x when the main columns are contiguous and 8-aligned, else eight clamped scalar loads
     const bool vec = !L.colmap && a.xt != VQLIN_F32 && (L.n_in & 7) == 0;
@@ -348,7 +348,7 @@ __global__ void __launch_bounds__(256) k_cs_finalize(Layer L, const float* __res
   const int i0 = blockIdx.x * 32;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   // the next grid may start its layer-only prologue; it waits for this grid before reading x
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  pdl_release();
   with_dtype(xt, [&](auto tag) {
     constexpr int XT = decltype(tag)::value;
     // sparse term of rows i0 + 4*warp .. +3
@@ -439,7 +439,7 @@ __global__ void __launch_bounds__(256) k_cs_finalize(Layer L, const float* __res
     if (L.rs && (t >> 5) < NB && i < L.n_out) rsc = __half2float(L.rs[i]);
   }
   // the planes are written by the preceding codebook-stationary grid
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  pdl_wait();
   {
     const int g = warp, r = lane, i = i0 + r;
     const size_t stride = (size_t)batch * L.n_out;
@@ -475,29 +475,12 @@ __global__ void __launch_bounds__(256) k_cs_finalize(Layer L, const float* __res
   }
 }
 
-// Both grids are launched as programmatic dependents of whatever precedes them on the stream.
-static cudaLaunchConfig_t pdl_config(dim3 grid, int threads, size_t smem, cudaStream_t s, cudaLaunchAttribute* attr) {
-  cudaLaunchConfig_t cfg = {};
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.gridDim = grid;
-  cfg.blockDim = dim3(threads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cfg;
-}
-
 template <int NB, int EPW>
 static cudaError_t launch_cfg(const Args& a, size_t smem, cudaStream_t s) {
   auto k = k_gemv_cs<NB, EPW>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  cudaLaunchAttribute attr[1];
-  const cudaLaunchConfig_t cfg = pdl_config(dim3(a.L.cs_P * a.L.cs_H), THREADS, smem, s, attr);
-  note_launches(1);
-  return cudaLaunchKernelEx(&cfg, k, a);
+  return launch_pdl(k, dim3(a.L.cs_P * a.L.cs_H), THREADS, smem, s, a);
 }
 
 }  // namespace csg
@@ -543,14 +526,12 @@ cudaError_t launch_gemv_cs(const Layer& L, const void* x, vqlin_dtype xt, int ba
     else e = launch_cfg<4, 2>(a, smem, s);
   }
   if (e != cudaSuccess) return e;
-  cudaLaunchAttribute attr[1];
-  const cudaLaunchConfig_t cfg = pdl_config(dim3((L.n_out + 31) / 32), 256, 0, s, attr);
   const float* planes = a.planes;
   const int P = L.cs_P;
-  note_launches(1);
-  if (NB == 1) e = cudaLaunchKernelEx(&cfg, k_cs_finalize<1>, L, planes, P, x, xt, batch, y, yt);
-  else if (NB == 2) e = cudaLaunchKernelEx(&cfg, k_cs_finalize<2>, L, planes, P, x, xt, batch, y, yt);
-  else e = cudaLaunchKernelEx(&cfg, k_cs_finalize<4>, L, planes, P, x, xt, batch, y, yt);
+  const dim3 fgrid((L.n_out + 31) / 32);
+  if (NB == 1) e = launch_pdl(k_cs_finalize<1>, fgrid, 256, 0, s, L, planes, P, x, xt, batch, y, yt);
+  else if (NB == 2) e = launch_pdl(k_cs_finalize<2>, fgrid, 256, 0, s, L, planes, P, x, xt, batch, y, yt);
+  else e = launch_pdl(k_cs_finalize<4>, fgrid, 256, 0, s, L, planes, P, x, xt, batch, y, yt);
   if (e == cudaSuccess) e = cudaGetLastError();
   *handled = (e == cudaSuccess);
   return e;

@@ -136,6 +136,9 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
       for (int i = threadIdx.x; i < L.k2 * COPIES; i += THREADS) cb2s[i] = __ldg(c2 + i / COPIES);
     }
   }
+  // x (and the accumulator) belong to the previous grid until it completes
+  pdl_wait();
+  pdl_release();
   // ---- outlier-block x' (fp32), once per CTA
   const int n_o = L.n_sub_o * 8;
   for (int i = threadIdx.x; i < BP * n_o; i += THREADS) {
@@ -217,6 +220,36 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
     const int ch0 = a.split ? task / n_rg : 0;
     const int ch1 = a.split ? ch0 + 1 : a.n_chunks;
     for (int i = threadIdx.x; i < a.rtt * 16 * 8 * NT; i += THREADS) red[i] = 0.f;
+    // sparse correction and outlier block of this thread's row first: their dependent loads
+    // overlap the MMA work below
+    const bool first_chunk = ch0 == 0;
+    const int rows = a.rtt * 16;
+    const int lanes_per_row = THREADS / rows;       // rows * lanes_per_row == THREADS
+    const int rl = threadIdx.x / lanes_per_row, sub = threadIdx.x - rl * lanes_per_row;
+    const int64_t row = (int64_t)rg * rows + rl;
+    const bool row_ok = row < L.n_out;
+    float spv[BP], ov[BP];
+#pragma unroll
+    for (int b = 0; b < BP; ++b) spv[b] = ov[b] = 0.f;
+    if (first_chunk && row_ok) {
+      if (L.nnz > 0) sparse_row_terms<BP>(L, a.x, a.xt, B, row, sub, lanes_per_row, spv);
+      for (int s = sub; s < L.n_sub_o; s += lanes_per_row) {
+        uint32_t f = read_field(L.codes_o + row * L.stride_o, s, L.bits_o);
+        uint4 u = __ldg(reinterpret_cast<const uint4*>(L.cbo) + f);
+        const __half2* h = reinterpret_cast<const __half2*>(&u);
+        float c[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) { float2 f2 = __half22float2(h[k]); c[2 * k] = f2.x; c[2 * k + 1] = f2.y; }
+#pragma unroll
+        for (int b = 0; b < BP; ++b)
+          if (b < B) {
+            float acc = ov[b];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) acc = fmaf(c[k], xo[b * n_o + s * 8 + k], acc);
+            ov[b] = acc;
+          }
+      }
+    }
     float d[NT][4];
 #pragma unroll
     for (int n = 0; n < NT; ++n) d[n][0] = d[n][1] = d[n][2] = d[n][3] = 0.f;
@@ -309,57 +342,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
       }
     }
     __syncthreads();
-    // ---- epilogue: (rtt*16 rows) x batch, sparse correction and outlier block
-    const bool first_chunk = ch0 == 0;
-    const int rows = a.rtt * 16;
-    const int lanes_per_row = THREADS / rows;       // rows * lanes_per_row == THREADS
-    const int rl = threadIdx.x / lanes_per_row, sub = threadIdx.x - rl * lanes_per_row;
-    const int64_t row = (int64_t)rg * rows + rl;
-    const bool row_ok = row < L.n_out;
+    // ---- epilogue: (rtt*16 rows) x batch, sparse correction and outlier block (computed above)
     {
-      float spv[BP], ov[BP];
-#pragma unroll
-      for (int b = 0; b < BP; ++b) spv[b] = ov[b] = 0.f;
-      if (first_chunk && row_ok) {
-        if (L.nnz > 0) {
-          const int e_end = L.row_ptr[row + 1];
-          for (int e0 = L.row_ptr[row] + sub; e0 < e_end; e0 += 8 * lanes_per_row) {
-            float dl[8];
-            int jj[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int e = e0 + u * lanes_per_row;
-              dl[u] = e < e_end ? L.delta[e] : 0.f;
-              jj[u] = e < e_end ? (L.col16 ? (int)L.col16[e] : L.col[e]) : 0;
-            }
-#pragma unroll
-            for (int b = 0; b < BP; ++b)
-              if (b < B) {
-                float xv[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) xv[u] = load_as_float(a.x, a.xt, (int64_t)b * L.n_in + jj[u]);
-#pragma unroll
-                for (int u = 0; u < 8; ++u) spv[b] = fmaf(dl[u], xv[u], spv[b]);
-              }
-          }
-        }
-        for (int s = sub; s < L.n_sub_o; s += lanes_per_row) {
-          uint32_t f = read_field(L.codes_o + row * L.stride_o, s, L.bits_o);
-          uint4 u = __ldg(reinterpret_cast<const uint4*>(L.cbo) + f);
-          const __half2* h = reinterpret_cast<const __half2*>(&u);
-          float c[8];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) { float2 f2 = __half22float2(h[k]); c[2 * k] = f2.x; c[2 * k + 1] = f2.y; }
-#pragma unroll
-          for (int b = 0; b < BP; ++b)
-            if (b < B) {
-              float acc = ov[b];
-#pragma unroll
-              for (int k = 0; k < 8; ++k) acc = fmaf(c[k], xo[b * n_o + s * 8 + k], acc);
-              ov[b] = acc;
-            }
-        }
-      }
       // reduce over the lanes of this row (they are consecutive threads)
 #pragma unroll
       for (int b = 0; b < BP; ++b) {
@@ -421,6 +405,9 @@ __global__ void __launch_bounds__(THREADS, 2) k_gemv_wt(Args a) {
       for (int i = threadIdx.x; i < L.k2 * COPIES; i += THREADS) cb2s[i] = __ldg(c2 + i / COPIES);
     }
   }
+  // x (and the accumulator) belong to the previous grid until it completes
+  pdl_wait();
+  pdl_release();
   const int n_o = L.n_sub_o * 8;
   for (int i = threadIdx.x; i < BP * n_o; i += THREADS) {
     int b = i / n_o, p = i - b * n_o;
@@ -490,28 +477,7 @@ __global__ void __launch_bounds__(THREADS, 2) k_gemv_wt(Args a) {
       float spv[BP], ov[BP];
 #pragma unroll
       for (int b = 0; b < BP; ++b) spv[b] = ov[b] = 0.f;
-      if (ok && L.nnz > 0) {
-        const int e_end = L.row_ptr[row + 1];
-        for (int e0 = L.row_ptr[row] + sub; e0 < e_end; e0 += 32) {
-          float dl[8];
-          int jj[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int e = e0 + 4 * u;
-            dl[u] = e < e_end ? L.delta[e] : 0.f;
-            jj[u] = e < e_end ? (L.col16 ? (int)L.col16[e] : L.col[e]) : 0;
-          }
-#pragma unroll
-          for (int b = 0; b < BP; ++b)
-            if (b < B) {
-              float xv[8];
-#pragma unroll
-              for (int u = 0; u < 8; ++u) xv[u] = load_as_float(a.x, a.xt, (int64_t)b * L.n_in + jj[u]);
-#pragma unroll
-              for (int u = 0; u < 8; ++u) spv[b] = fmaf(dl[u], xv[u], spv[b]);
-            }
-        }
-      }
+      if (ok && L.nnz > 0) sparse_row_terms<BP>(L, a.x, a.xt, B, row, sub, 4, spv);
       if (ok) {
         for (int so = sub; so < L.n_sub_o; so += 4) {
           uint32_t f = read_field(L.codes_o + row * L.stride_o, so, L.bits_o);
@@ -634,9 +600,7 @@ static cudaError_t launch_wt_cfg(const Args& args, size_t smem, int grid, cudaSt
   auto k = k_gemv_wt<NT, W, CB_SMEM, COPIES>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  note_launches(1);
-  k<<<grid, THREADS, smem, s>>>(args);
-  return cudaGetLastError();
+  return launch_pdl(k, dim3(grid), THREADS, smem, s, args);
 }
 
 template <int NT, int W>
@@ -662,6 +626,8 @@ static cudaError_t launch_wt_nt(const Args& args, bool cb_smem, int copies, size
 }
 
 __global__ void k_finalize(const float* __restrict__ acc, int64_t n, void* __restrict__ y, vqlin_dtype yt) {
+  pdl_wait();
+  pdl_release();
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
     store_from_float(y, yt, i, acc[i]);
 }
@@ -671,9 +637,7 @@ static cudaError_t launch_cfg(const Args& args, size_t smem, int grid, cudaStrea
   auto k = k_gemv_tc<NT, W, CB_SMEM, COPIES>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  note_launches(1);
-  k<<<grid, THREADS, smem, s>>>(args);
-  return cudaGetLastError();
+  return launch_pdl(k, dim3(grid), THREADS, smem, s, args);
 }
 
 template <int NT, int W>
@@ -709,6 +673,15 @@ size_t gemv_workspace_bytes(const Layer& L, int batch) {
   const size_t cs = gemv_cs_workspace_bytes(L, batch);
   return acc > cs ? acc : cs;
 }
+
+// Clears an fp32 accumulator once the previous grid has completed.
+__global__ void k_zero(float* __restrict__ p, int64_t n) {
+  pdl_wait();
+  pdl_release();
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) p[i] = 0.f;
+}
+
+static int small_grid(int64_t n) { return (int)((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024); }
 
 // Plan and launch.  acc_ws: caller workspace for split accumulation (may be null).
 cudaError_t launch_gemv_tc(const Layer& L, const void* x, vqlin_dtype xt, int batch, void* y, vqlin_dtype yt,
@@ -753,8 +726,9 @@ cudaError_t launch_gemv_tc(const Layer& L, const void* x, vqlin_dtype xt, int ba
   const int n_rt = (L.n_out + 15) / 16;
   const int n_rg = (n_rt + a.rtt - 1) / a.rtt;
   // ---- warp-task kernel: needs an fp32 accumulator (y itself, or the caller's workspace)
-  //      and x' for every column next to the codebooks
-  {
+  //      and x' for every column next to the codebooks.  When one block task already
+  //      covers every column, the block-task kernel below writes y in a single grid.
+  if (a.n_chunks > 1) {
     float* acc = nullptr;
     if (yt == VQLIN_F32) acc = reinterpret_cast<float*>(y);
     else if (ws && ws_bytes >= gemv_workspace_bytes(L, batch)) acc = reinterpret_cast<float*>(ws);
@@ -776,7 +750,8 @@ cudaError_t launch_gemv_tc(const Layer& L, const void* x, vqlin_dtype xt, int ba
       const int per_sm = (int)(smem_max / (wsmem + 1024)) >= 2 ? 2 : 1;
       int grid = sms * per_sm;
       if (grid > (total + WARPS - 1) / WARPS) grid = (total + WARPS - 1) / WARPS;
-      cudaError_t e = cudaMemsetAsync(acc, 0, (size_t)batch * L.n_out * 4, s);
+      cudaError_t e = launch_pdl(k_zero, dim3(small_grid((int64_t)batch * L.n_out)), 256, 0, s, acc,
+                                 (int64_t)batch * L.n_out);
       if (e != cudaSuccess) return e;
       if (NT == 1) e = launch_wt_nt<1>(w, wcb, wcopies, wsmem, grid, s);
       else if (NT == 2) e = launch_wt_nt<2>(w, wcb, wcopies, wsmem, grid, s);
@@ -784,9 +759,7 @@ cudaError_t launch_gemv_tc(const Layer& L, const void* x, vqlin_dtype xt, int ba
       if (e != cudaSuccess) return e;
       if (yt != VQLIN_F32) {
         int64_t n = (int64_t)batch * L.n_out;
-        note_launches(1);
-        k_finalize<<<(int)((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024), 256, 0, s>>>(acc, n, y, yt);
-        e = cudaGetLastError();
+        e = launch_pdl(k_finalize, dim3(small_grid(n)), 256, 0, s, (const float*)acc, n, y, yt);
       }
       *handled = (e == cudaSuccess);
       return e;
@@ -806,7 +779,7 @@ cudaError_t launch_gemv_tc(const Layer& L, const void* x, vqlin_dtype xt, int ba
   if (grid > n_tasks) grid = n_tasks;
   cudaError_t e;
   if (a.split) {
-    e = cudaMemsetAsync(a.acc, 0, (size_t)batch * L.n_out * 4, s);
+    e = launch_pdl(k_zero, dim3(small_grid((int64_t)batch * L.n_out)), 256, 0, s, a.acc, (int64_t)batch * L.n_out);
     if (e != cudaSuccess) return e;
   }
   if (NT == 1) e = launch_nt<1>(a, cb_smem, copies, smem, grid, s);
@@ -815,9 +788,7 @@ cudaError_t launch_gemv_tc(const Layer& L, const void* x, vqlin_dtype xt, int ba
   if (e != cudaSuccess) return e;
   if (a.split && yt != VQLIN_F32) {
     int64_t n = (int64_t)batch * L.n_out;
-    note_launches(1);
-    k_finalize<<<(int)((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024), 256, 0, s>>>(a.acc, n, y, yt);
-    e = cudaGetLastError();
+    e = launch_pdl(k_finalize, dim3(small_grid(n)), 256, 0, s, (const float*)a.acc, n, y, yt);
   }
   *handled = (e == cudaSuccess);
   return e;

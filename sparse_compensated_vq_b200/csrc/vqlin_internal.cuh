@@ -136,6 +136,65 @@ __device__ __forceinline__ uint32_t read_field(const uint8_t* row, int64_t s, in
   return w >= 32 ? (uint32_t)v : (uint32_t)(v & ((1ull << w) - 1ull));
 }
 
+// Fused sparse term of one row, sum_e delta_e * x[b][col_e], over the row's CSR entries
+// sub, sub + stride, ... (the caller reduces over its `stride` lanes).  Eight entries per
+// round with clamped indices, so the eight loads of each kind issue together; x is read with
+// its compile-time dtype.
+template <int BP>
+__device__ __forceinline__ void sparse_row_terms(const Layer& L, const void* x, vqlin_dtype xt, int B, int64_t row,
+                                                 int sub, int stride, float* spv) {
+  const int e_beg = L.row_ptr[row], e_end = L.row_ptr[row + 1];
+  with_dtype(xt, [&](auto tag) {
+    constexpr int XT = decltype(tag)::value;
+    for (int e0 = e_beg + sub; e0 < e_end; e0 += 8 * stride) {
+      float dl[8];
+      int jj[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int e = min(e0 + u * stride, e_end - 1);
+        dl[u] = L.delta[e];
+        jj[u] = L.col16 ? (int)L.col16[e] : L.col[e];
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) if (e0 + u * stride >= e_end) dl[u] = 0.f;
+#pragma unroll
+      for (int b = 0; b < BP; ++b)
+        if (b < B) {
+          float xv[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) xv[u] = ldx<XT>(x, (int64_t)b * L.n_in + jj[u]);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) spv[b] = fmaf(dl[u], xv[u], spv[b]);
+        }
+    }
+  });
+}
+
+// Programmatic dependent launch.  Decode kernels are launched so that they may start
+// while the previous grid on the stream is still running; everything they do before
+// pdl_wait() reads only the layer (immutable after create) and writes only shared memory.
+// pdl_wait() returns once the previous grid has completed and its writes are visible;
+// pdl_release() then lets the next grid start its own layer-only prologue (that grid
+// still waits for this one before it reads anything this one writes).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <class K, class... A>
+cudaError_t launch_pdl(K kernel, dim3 grid, int threads, size_t smem, cudaStream_t s, A... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  note_launches(1);
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 }  // namespace vqlin
 
 // The public handle.
