@@ -170,6 +170,67 @@ __device__ __forceinline__ void sparse_row_terms(const Layer& L, const void* x, 
   });
 }
 
+// The same term split in two for a kernel's layer-only prologue: sparse_prefetch reads the
+// row's CSR bounds and its first eight entries of this lane (layer data, before the kernel
+// waits for the previous grid); sparse_finish gathers x for them and walks the rest.
+struct SparsePre {
+  int e0, e_end;
+  float dl[8];
+  int jj[8];
+};
+
+__device__ __forceinline__ void sparse_prefetch(const Layer& L, int64_t row, int sub, int stride, SparsePre& p) {
+  p.e0 = L.row_ptr[row] + sub;
+  p.e_end = L.row_ptr[row + 1];
+  const int last = max(p.e_end - 1, 0);
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int e = min(p.e0 + u * stride, last);
+    p.dl[u] = L.delta[e];
+    p.jj[u] = L.col16 ? (int)L.col16[e] : L.col[e];
+  }
+#pragma unroll
+  for (int u = 0; u < 8; ++u) if (p.e0 + u * stride >= p.e_end) { p.dl[u] = 0.f; p.jj[u] = 0; }
+}
+
+template <int BP>
+__device__ __forceinline__ void sparse_finish(const Layer& L, const void* x, vqlin_dtype xt, int B, const SparsePre& p,
+                                              int stride, float* spv) {
+  with_dtype(xt, [&](auto tag) {
+    constexpr int XT = decltype(tag)::value;
+#pragma unroll
+    for (int b = 0; b < BP; ++b)
+      if (b < B) {
+        float xv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) xv[u] = ldx<XT>(x, (int64_t)b * L.n_in + p.jj[u]);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) spv[b] = fmaf(p.dl[u], xv[u], spv[b]);
+      }
+    for (int e0 = p.e0 + 8 * stride; e0 < p.e_end; e0 += 8 * stride) {
+      float dl[8];
+      int jj[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int e = min(e0 + u * stride, p.e_end - 1);
+        dl[u] = L.delta[e];
+        jj[u] = L.col16 ? (int)L.col16[e] : L.col[e];
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) if (e0 + u * stride >= p.e_end) dl[u] = 0.f;
+#pragma unroll
+      for (int b = 0; b < BP; ++b)
+        if (b < B) {
+          float xv[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) xv[u] = ldx<XT>(x, (int64_t)b * L.n_in + jj[u]);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) spv[b] = fmaf(dl[u], xv[u], spv[b]);
+        }
+    }
+  });
+}
+
 // Programmatic dependent launch.  Decode kernels are launched so that they may start
 // while the previous grid on the stream is still running; everything they do before
 // pdl_wait() reads only the layer (immutable after create) and writes only shared memory.
