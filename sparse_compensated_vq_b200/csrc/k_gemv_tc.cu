@@ -136,9 +136,47 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
       for (int i = threadIdx.x; i < L.k2 * COPIES; i += THREADS) cb2s[i] = __ldg(c2 + i / COPIES);
     }
   }
+  // ---- layer-only prefetch for this block's first task, before the wait: the index words of
+  //      each warp's first (row tile, kernel slab) and the CSR bounds and first entries of each
+  //      thread's epilogue row
+  const int n_rt = (L.n_out + 15) / 16;
+  const int n_rg = (n_rt + a.rtt - 1) / a.rtt;
+  const int n_tasks = a.split ? n_rg * a.n_chunks : n_rg;
+  const int my_rt_local = warp / a.ks;            // which of the task's row tiles this warp serves
+  const int my_ks = warp - my_rt_local * a.ks;    // which kernel slab of the chunk
+  const bool warp_active = my_rt_local < a.rtt;
+  const int rows = a.rtt * 16;
+  const int lanes_per_row = THREADS / rows;       // rows * lanes_per_row == THREADS
+  const int rl = threadIdx.x / lanes_per_row, sub = threadIdx.x - rl * lanes_per_row;
+  constexpr int NWORDS = (2 * W / NT + 3) / 4 + 1;
+  const int task0 = blockIdx.x;
+  uint32_t pw0[NWORDS], pw1[NWORDS];
+  pw0[NWORDS - 1] = pw1[NWORDS - 1] = 0;
+  SparsePre spre;
+  bool spre_ok = false;
+  if (task0 < n_tasks) {
+    const int rg0 = a.split ? task0 % n_rg : task0;
+    const int ch00 = a.split ? task0 / n_rg : 0;
+    const int rt0 = rg0 * a.rtt + my_rt_local, kslab0 = ch00 * a.ks + my_ks;
+    if (warp_active && rt0 < n_rt && kslab0 < a.n_kslabs) {
+      const int ls = kslab0 / NT, ps0 = (kslab0 - ls * NT) * PS;
+      const uint8_t* blk0 = L.tcodes + ((int64_t)rt0 * 16 + g) * L.tstride + (int64_t)ls * (8 * W) + t * (2 * W) + ps0 * W / 8;
+      load_sub<W, NT>(blk0, pw0);
+      load_sub<W, NT>(blk0 + 8 * L.tstride, pw1);
+    }
+    const int64_t row0 = (int64_t)rg0 * rows + rl;
+    if (ch00 == 0 && row0 < L.n_out && L.nnz > 0) {
+      sparse_prefetch(L, row0, sub, lanes_per_row, spre);
+      spre_ok = true;
+    }
+  }
   // x (and the accumulator) belong to the previous grid until it completes
   pdl_wait();
   pdl_release();
+  float spv0[BP];
+#pragma unroll
+  for (int b = 0; b < BP; ++b) spv0[b] = 0.f;
+  if (spre_ok) sparse_finish<BP>(L, a.x, a.xt, B, spre, lanes_per_row, spv0);
   // ---- outlier-block x' (fp32), once per CTA
   const int n_o = L.n_sub_o * 8;
   for (int i = threadIdx.x; i < BP * n_o; i += THREADS) {
@@ -200,9 +238,6 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
     }
   };
 
-  const int n_rt = (L.n_out + 15) / 16;
-  const int n_rg = (n_rt + a.rtt - 1) / a.rtt;
-  const int n_tasks = a.split ? n_rg * a.n_chunks : n_rg;
   const int chunk_cols = a.ks * KSV * 8;
   int staged = -1;
   if (a.xs_all) {
@@ -211,28 +246,20 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
   }
   __syncthreads();
 
-  const int my_rt_local = warp / a.ks;            // which of the task's row tiles this warp serves
-  const int my_ks = warp - my_rt_local * a.ks;    // which kernel slab of the chunk
-  const bool warp_active = my_rt_local < a.rtt;
-
   for (int task = blockIdx.x; task < n_tasks; task += gridDim.x) {
     const int rg = a.split ? task % n_rg : task;
     const int ch0 = a.split ? task / n_rg : 0;
     const int ch1 = a.split ? ch0 + 1 : a.n_chunks;
     for (int i = threadIdx.x; i < a.rtt * 16 * 8 * NT; i += THREADS) red[i] = 0.f;
-    // sparse correction and outlier block of this thread's row first: their dependent loads
-    // overlap the MMA work below
+    // sparse correction (prefetched for the first task) and outlier block of this thread's row
     const bool first_chunk = ch0 == 0;
-    const int rows = a.rtt * 16;
-    const int lanes_per_row = THREADS / rows;       // rows * lanes_per_row == THREADS
-    const int rl = threadIdx.x / lanes_per_row, sub = threadIdx.x - rl * lanes_per_row;
     const int64_t row = (int64_t)rg * rows + rl;
     const bool row_ok = row < L.n_out;
     float spv[BP], ov[BP];
 #pragma unroll
-    for (int b = 0; b < BP; ++b) spv[b] = ov[b] = 0.f;
+    for (int b = 0; b < BP; ++b) { spv[b] = task == task0 ? spv0[b] : 0.f; ov[b] = 0.f; }
     if (first_chunk && row_ok) {
-      if (L.nnz > 0) sparse_row_terms<BP>(L, a.x, a.xt, B, row, sub, lanes_per_row, spv);
+      if (L.nnz > 0 && task != task0) sparse_row_terms<BP>(L, a.x, a.xt, B, row, sub, lanes_per_row, spv);
       for (int s = sub; s < L.n_sub_o; s += lanes_per_row) {
         uint32_t f = read_field(L.codes_o + row * L.stride_o, s, L.bits_o);
         uint4 u = __ldg(reinterpret_cast<const uint4*>(L.cbo) + f);
@@ -281,14 +308,17 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
           bf[ps][n] = v;
         }
       }
-      // this kernel slab's fields of rows g and g+8 of the row tile
-      constexpr int NWORDS = (2 * W / NT + 3) / 4 + 1;
+      // this kernel slab's fields of rows g and g+8 of the row tile (prefetched for the first one)
       uint32_t w0[NWORDS], w1[NWORDS];
-      w0[NWORDS - 1] = w1[NWORDS - 1] = 0;
-      const int64_t R0 = (int64_t)rt * 16 + g;
-      const uint8_t* blk0 = L.tcodes + R0 * L.tstride + (int64_t)ls * (8 * W) + t * (2 * W) + ps0 * W / 8;
-      load_sub<W, NT>(blk0, w0);
-      load_sub<W, NT>(blk0 + 8 * L.tstride, w1);
+      if (task == task0 && ch == ch0) {
+#pragma unroll
+        for (int i = 0; i < NWORDS; ++i) { w0[i] = pw0[i]; w1[i] = pw1[i]; }
+      } else {
+        w0[NWORDS - 1] = w1[NWORDS - 1] = 0;
+        const uint8_t* blk0 = L.tcodes + ((int64_t)rt * 16 + g) * L.tstride + (int64_t)ls * (8 * W) + t * (2 * W) + ps0 * W / 8;
+        load_sub<W, NT>(blk0, w0);
+        load_sub<W, NT>(blk0 + 8 * L.tstride, w1);
+      }
       // gathers of G pair-steps are issued before their MMAs (hides L2 / shared latency)
       constexpr int G = (W >= 24 || PS < 8) ? (PS < 4 ? PS : 4) : 8;
       static_assert(PS % G == 0 && G <= PS, "pair-step batches must tile the kernel slab");
