@@ -119,6 +119,98 @@ __global__ void k_convert_f16(const unsigned short* __restrict__ X, vqlin_dtype 
   }
 }
 
+// bf16 -> fp16, eight elements per thread with 16-byte loads and stores (n % 8 == 0, both
+// buffers 16-byte aligned).
+__global__ void k_convert_bf16_f16_x8(const uint4* __restrict__ X, int64_t n8, uint4* __restrict__ out) {
+  for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < n8; t += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 v = __ldg(X + t);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float lo = __uint_as_float(w[k] << 16), hi = __uint_as_float(w[k] & 0xFFFF0000u);   // bf16 -> fp32 exact
+      o[k] = (uint32_t)__half_as_ushort(__float2half_rn(lo)) | ((uint32_t)__half_as_ushort(__float2half_rn(hi)) << 16);
+    }
+    out[t] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// Exact dequantisation on the codebook-stationary layout (single-stage codebook, no outlier
+// block, W rows 16-byte aligned).  Block (p, h) holds codebook slice p as 8 interleaved
+// copies, the column scales as fp32 and the row scales of half h; every entry (row, position,
+// index) of its bucket becomes one 16-byte store of eight fp16 weights.
+//
+// Exactness in fp32: a centroid element C and the row scale r are fp16, so C*r has at most
+// 22 significant bits and is exact in fp32.  The product with the column scale is taken
+// rounded toward zero with its exact error from an FMA, and the last bit is forced to 1 when
+// inexact (round-to-odd, Boldo & Melquiond, IEEE TC 2008); a 24-bit round-to-odd value
+// rounds to the 11-bit fp16 exactly as the real value would.  Null entries are skipped.
+__device__ __forceinline__ float round_to_odd_mul_f32(float a, float b) {
+  float p = __fmul_rz(a, b);
+  const float err = fmaf(a, b, -p);
+  if (err != 0.f) p = __int_as_float(__float_as_int(p) | 1);
+  return p;
+}
+
+template <int EPW>
+__global__ void __launch_bounds__(512, 1) k_dequant_cs(Layer L, __half* __restrict__ W, int64_t ldw) {
+  constexpr int THREADS = 512, COPIES = 8;
+  constexpr int SLOT = EPW == 3 ? 21 : 32;
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int H = L.cs_H, E = L.cs_E, RPP = L.cs_rpp;
+  const int c = blockIdx.x;
+  const int p = c / H, h = c - p * H;
+  const int row0 = h * RPP;
+  const int nrows = min(RPP, L.n_out - row0);
+  const int slice0 = p * E, E_p = max(0, min(E, L.k1 - slice0));
+  uint4* cbs = reinterpret_cast<uint4*>(smem);                                        // [E + 1][8]
+  float* cf = reinterpret_cast<float*>(smem + (size_t)(E + 1) * COPIES * 16);         // [n_sub * 8]
+  float* rf = cf + (size_t)L.n_sub * 8;                                               // [RPP]
+  const int rot = threadIdx.x & (COPIES - 1);
+  for (int k = threadIdx.x; k < E_p; k += THREADS) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(L.cb1) + slice0 + k);
+#pragma unroll
+    for (int cc = 0; cc < COPIES; ++cc) cbs[k * COPIES + ((cc + rot) & (COPIES - 1))] = v;
+  }
+  for (int j = threadIdx.x; j < L.n_sub * 8; j += THREADS) cf[j] = (L.cs && j < L.n_main) ? __half2float(L.cs[j]) : 1.f;
+  for (int r = threadIdx.x; r < nrows; r += THREADS) rf[r] = L.rs ? __half2float(L.rs[row0 + r]) : 1.f;
+  __syncthreads();
+  const uint32_t lmask = (1u << L.cs_local_bits) - 1u;
+  const uint64_t emask = (1ull << L.cs_ebits) - 1ull;
+  const int lbits = L.cs_local_bits;
+  const int64_t w_begin = L.cs_start[c];
+  const int n_words = (int)(L.cs_start[c + 1] - w_begin);
+  const bool has_cs = L.cs != nullptr;
+  for (int wi = threadIdx.x; wi < n_words; wi += THREADS) {
+    const uint64_t wv = __ldg(reinterpret_cast<const unsigned long long*>(L.cs_words) + w_begin + wi);
+    const int s = __ldg(L.cs_wpos + w_begin + wi);
+    const float4 c0 = *reinterpret_cast<const float4*>(cf + s * 8), c1 = *reinterpret_cast<const float4*>(cf + s * 8 + 4);
+    const float cc8[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+    for (int u = 0; u < EPW; ++u) {
+      const uint32_t ent = (uint32_t)((wv >> (u * SLOT)) & emask);
+      const uint32_t k = ent & lmask;
+      if (k == (uint32_t)E) continue;                        // null entry
+      const int row_l = (int)(ent >> lbits);
+      const uint4 cen = cbs[k * COPIES + (threadIdx.x & (COPIES - 1))];
+      const __half* ch = reinterpret_cast<const __half*>(&cen);
+      const float r = rf[row_l];
+      uint32_t o[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float v2[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float a = __half2float(ch[2 * q + e]) * r;   // exact
+          v2[e] = has_cs ? round_to_odd_mul_f32(a, cc8[2 * q + e]) : a;
+        }
+        o[q] = (uint32_t)__half_as_ushort(__float2half_rn(v2[0])) | ((uint32_t)__half_as_ushort(__float2half_rn(v2[1])) << 16);
+      }
+      *reinterpret_cast<uint4*>(W + (int64_t)(row0 + row_l) * ldw + (int64_t)s * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+}
+
 static int grid_for(int64_t work, int threads) {
   int64_t g = (work + threads - 1) / threads;
   if (g > 148 * 32) g = 148 * 32;
@@ -136,6 +228,26 @@ cudaError_t launch_unpack(const Layer& L, int which, uint32_t* out, cudaStream_t
 
 cudaError_t launch_dequant(const Layer& L, __half* W, int64_t ldw, cudaStream_t s) {
   int64_t work = (int64_t)L.n_out * (L.n_sub + L.n_sub_o);
+  const bool cs_ok = L.cs_words && !L.colmap && L.k2 == 0 && (ldw & 7) == 0 && (L.n_main & 7) == 0 &&
+                     (reinterpret_cast<uintptr_t>(W) & 15) == 0;
+  const size_t cs_smem = (size_t)(L.cs_E + 1) * 8 * 16 + (size_t)L.n_sub * 8 * 4 + (size_t)L.cs_rpp * 4;
+  if (cs_ok && cs_smem <= 227 * 1024) {
+    cudaError_t e;
+    if (L.cs_epw == 3) {
+      e = cudaFuncSetAttribute(k_dequant_cs<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cs_smem);
+      if (e != cudaSuccess) return e;
+      note_launches(1);
+      k_dequant_cs<3><<<L.cs_P * L.cs_H, 512, cs_smem, s>>>(L, W, ldw);
+    } else {
+      e = cudaFuncSetAttribute(k_dequant_cs<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cs_smem);
+      if (e != cudaSuccess) return e;
+      note_launches(1);
+      k_dequant_cs<2><<<L.cs_P * L.cs_H, 512, cs_smem, s>>>(L, W, ldw);
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    work = 0;                                   // the main block is done (no outlier block here)
+  }
   if (work > 0) {
     note_launches(1);
     if (L.d == 8) k_dequant_body<8><<<grid_for(work, 256), 256, 0, s>>>(L, W, ldw);
@@ -152,6 +264,13 @@ cudaError_t launch_dequant(const Layer& L, __half* W, int64_t ldw, cudaStream_t 
 }
 
 cudaError_t launch_convert_to_f16(const void* X, vqlin_dtype xt, int64_t n, __half* out, cudaStream_t s) {
+  if (xt == VQLIN_BF16 && (n & 7) == 0 && (reinterpret_cast<uintptr_t>(X) & 15) == 0 &&
+      (reinterpret_cast<uintptr_t>(out) & 15) == 0) {
+    note_launches(1);
+    k_convert_bf16_f16_x8<<<grid_for(n / 8, 256), 256, 0, s>>>(reinterpret_cast<const uint4*>(X), n / 8,
+                                                              reinterpret_cast<uint4*>(out));
+    return cudaGetLastError();
+  }
   note_launches(1);
   k_convert_f16<<<grid_for(n, 256), 256, 0, s>>>(reinterpret_cast<const unsigned short*>(X), xt, n, out);
   return cudaGetLastError();

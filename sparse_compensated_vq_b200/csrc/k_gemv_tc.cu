@@ -110,6 +110,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
   constexpr int PS = 16 / NT;            // pair-steps (4 sub-vectors each) per kernel slab
   constexpr int KSV = 4 * PS;            // sub-vectors per kernel slab
   constexpr int BP = 4 * NT;             // batch slots
+  constexpr int ACC = NT == 1 ? 4 : 2;   // independent MMA accumulator sets
   const Layer& L = a.L;
   extern __shared__ __align__(16) unsigned char smem[];
   // ---- shared memory carve-up
@@ -154,6 +155,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
   pw0[NWORDS - 1] = pw1[NWORDS - 1] = 0;
   SparsePre spre;
   bool spre_ok = false;
+  float rsc0 = 1.f;                               // row scale of the first task's epilogue row
   if (task0 < n_tasks) {
     const int rg0 = a.split ? task0 % n_rg : task0;
     const int ch00 = a.split ? task0 / n_rg : 0;
@@ -165,6 +167,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
       load_sub<W, NT>(blk0 + 8 * L.tstride, pw1);
     }
     const int64_t row0 = (int64_t)rg0 * rows + rl;
+    if (L.rs && row0 < L.n_out) rsc0 = __half2float(L.rs[row0]);
     if (ch00 == 0 && row0 < L.n_out && L.nnz > 0) {
       sparse_prefetch(L, row0, sub, lanes_per_row, spre);
       spre_ok = true;
@@ -277,9 +280,12 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
           }
       }
     }
-    float d[NT][4];
+    // ACC independent accumulator sets, so consecutive MMAs do not wait on each other
+    float dacc[ACC][NT][4];
 #pragma unroll
-    for (int n = 0; n < NT; ++n) d[n][0] = d[n][1] = d[n][2] = d[n][3] = 0.f;
+    for (int q = 0; q < ACC; ++q)
+#pragma unroll
+      for (int n = 0; n < NT; ++n) dacc[q][n][0] = dacc[q][n][1] = dacc[q][n][2] = dacc[q][n][3] = 0.f;
     const int rt = rg * a.rtt + my_rt_local;
     for (int ch = ch0; ch < ch1; ++ch) {
       if (!a.xs_all && staged != ch) {
@@ -349,16 +355,27 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
         for (int j = 0; j < G; ++j) {
 #pragma unroll
           for (int n = 0; n < NT; ++n) {
-            mma16816(d[n], c0[j].x, c1[j].x, c0[j].y, c1[j].y, bf[p0 + j][n].x, bf[p0 + j][n].y);
-            mma16816(d[n], c0[j].z, c1[j].z, c0[j].w, c1[j].w, bf[p0 + j][n].z, bf[p0 + j][n].w);
+            const int q = (j % (ACC / 2)) * 2;
+            mma16816(dacc[q][n], c0[j].x, c1[j].x, c0[j].y, c1[j].y, bf[p0 + j][n].x, bf[p0 + j][n].y);
+            mma16816(dacc[q + 1][n], c0[j].z, c1[j].z, c0[j].w, c1[j].w, bf[p0 + j][n].z, bf[p0 + j][n].w);
             if (L.k2) {
-              mma16816(d[n], e0[j].x, e1[j].x, e0[j].y, e1[j].y, bf[p0 + j][n].x, bf[p0 + j][n].y);
-              mma16816(d[n], e0[j].z, e1[j].z, e0[j].w, e1[j].w, bf[p0 + j][n].z, bf[p0 + j][n].w);
+              mma16816(dacc[q][n], e0[j].x, e1[j].x, e0[j].y, e1[j].y, bf[p0 + j][n].x, bf[p0 + j][n].y);
+              mma16816(dacc[q + 1][n], e0[j].z, e1[j].z, e0[j].w, e1[j].w, bf[p0 + j][n].z, bf[p0 + j][n].w);
             }
           }
         }
       }
     }
+    float d[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float v = dacc[0][n][k];
+#pragma unroll
+        for (int q = 1; q < ACC; ++q) v += dacc[q][n][k];
+        d[n][k] = v;
+      }
     // ---- reduce the warps' D fragments: red[rt_local][row][col]
     if (warp_active) {
       float* r0 = red + ((size_t)my_rt_local * 16 + g) * (8 * NT);
@@ -382,7 +399,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
           ov[b] += __shfl_xor_sync(0xffffffffu, ov[b], o);
         }
       }
-      const float rsc = (L.rs && row_ok) ? __half2float(L.rs[row]) : 1.f;
+      const float rsc = task == task0 ? rsc0 : ((L.rs && row_ok) ? __half2float(L.rs[row]) : 1.f);
       const float* rr = red + (size_t)rl * (8 * NT);
 #pragma unroll
       for (int b = 0; b < BP; ++b) {
@@ -415,6 +432,7 @@ __global__ void __launch_bounds__(THREADS, 2) k_gemv_wt(Args a) {
   constexpr int PS = 16 / NT;
   constexpr int KSV = 4 * PS;
   constexpr int BP = 4 * NT;
+  constexpr int ACC = NT == 1 ? 4 : 2;   // independent MMA accumulator sets
   const Layer& L = a.L;
   extern __shared__ __align__(16) unsigned char smem[];
   uint4* cb1s = reinterpret_cast<uint4*>(smem);
@@ -549,9 +567,12 @@ __global__ void __launch_bounds__(THREADS, 2) k_gemv_wt(Args a) {
     load_sub<W, NT>(blk0 + 8 * L.tstride, w1);
     const float r0 = (L.rs && R0 < L.n_out) ? __half2float(L.rs[R0]) : 1.f;
     const float r1 = (L.rs && R0 + 8 < L.n_out) ? __half2float(L.rs[R0 + 8]) : 1.f;
-    float d[NT][4];
+    // ACC independent accumulator sets, so consecutive MMAs do not wait on each other
+    float dacc[ACC][NT][4];
 #pragma unroll
-    for (int n = 0; n < NT; ++n) d[n][0] = d[n][1] = d[n][2] = d[n][3] = 0.f;
+    for (int q = 0; q < ACC; ++q)
+#pragma unroll
+      for (int n = 0; n < NT; ++n) dacc[q][n][0] = dacc[q][n][1] = dacc[q][n][2] = dacc[q][n][3] = 0.f;
     const int col_base = kslab * KSV * 8;
     // gathers per batch: never more than the slab's pair-steps (PS is 4 when NT = 4)
     constexpr int G = ((W >= 24) ? 4 : 8) < PS ? ((W >= 24) ? 4 : 8) : PS;
@@ -589,15 +610,26 @@ __global__ void __launch_bounds__(THREADS, 2) k_gemv_wt(Args a) {
           else { part_lo = n / (NT / 2); bb = (n % (NT / 2)) * 8 + g; }
           uint4 bv = make_uint4(0, 0, 0, 0);
           if (bb < B) bv = *reinterpret_cast<const uint4*>((part_lo ? xl : xh) + (size_t)bb * a.xs_cols + col);
-          mma16816(d[n], c0[j].x, c1[j].x, c0[j].y, c1[j].y, bv.x, bv.y);
-          mma16816(d[n], c0[j].z, c1[j].z, c0[j].w, c1[j].w, bv.z, bv.w);
+          const int q = (j % (ACC / 2)) * 2;
+          mma16816(dacc[q][n], c0[j].x, c1[j].x, c0[j].y, c1[j].y, bv.x, bv.y);
+          mma16816(dacc[q + 1][n], c0[j].z, c1[j].z, c0[j].w, c1[j].w, bv.z, bv.w);
           if (L.k2) {
-            mma16816(d[n], e0[j].x, e1[j].x, e0[j].y, e1[j].y, bv.x, bv.y);
-            mma16816(d[n], e0[j].z, e1[j].z, e0[j].w, e1[j].w, bv.z, bv.w);
+            mma16816(dacc[q][n], e0[j].x, e1[j].x, e0[j].y, e1[j].y, bv.x, bv.y);
+            mma16816(dacc[q + 1][n], e0[j].z, e1[j].z, e0[j].w, e1[j].w, bv.z, bv.w);
           }
         }
       }
     }
+    float d[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float v = dacc[0][n][k];
+#pragma unroll
+        for (int q = 1; q < ACC; ++q) v += dacc[q][n][k];
+        d[n][k] = v;
+      }
     // hi + lo, times the row scale, into the accumulator
     if (NT == 1) {
       // columns 0-3 hold hi of batches 0-3, columns 4-7 lo: lanes t and t^2 pair up
