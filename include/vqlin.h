@@ -247,9 +247,20 @@ vqlin_status vqlin_unpack_indices(const vqlin_handle* h, int32_t which, uint32_t
  * every wait (1 s); when one gives up it records a code, skips its remaining
  * work and returns, so the context stays usable.  This call synchronises the
  * current device, returns the recorded code in *code (0 = none; 1-5 = the
- * GEMM pipeline wait that expired) and clears it.  No counterpart on the pages.
+ * GEMM pipeline wait that expired; 6 = the decode entry-stream wait; 7 = the
+ * self-test below) and clears it.  No counterpart on the pages.
  */
 vqlin_status vqlin_device_error(int32_t* code);
+
+/*
+ * Failure-detection self-test.  Launches on `stream` one thread that waits on a
+ * shared-memory mbarrier nothing completes, bounded by `limit_us` microseconds
+ * (1..1,000,000) of %globaltimer, exactly like the decode kernel's entry-stream
+ * wait.  When the limit passes the kernel records code 7 and returns, so a
+ * following vqlin_device_error() reports 7 and the context stays usable.  No
+ * counterpart on the pages.
+ */
+vqlin_status vqlin_selftest_wait_timeout(int32_t limit_us, void* stream);
 
 /*
  * Number of kernels this library has enqueued in this process so far, over

@@ -15,7 +15,9 @@
 //
 // A block holds its slice as 8 interleaved copies (entry k of copy c at k*8+c, so
 // the eight lanes of a quarter-warp, which read copies 0..7, always hit eight
-// different bank groups), x' = c (.) x for every position in fp32, and a
+// different bank groups; 4 copies, half the conflict-free width, when 8 would leave no room
+// for the whole entry stream next to a batch of 3-4), x' = c (.) x for every position in
+// fp32, and a
 // shared-memory accumulator for the rows of its half.  Its entry words and their
 // positions arrive by bulk asynchronous copies while it stages the rest.  Each
 // lane then takes one word (EPW entries of one position) at a time: x'[s] is a
@@ -46,7 +48,6 @@ namespace csg {
 
 constexpr int WARPS = 16;
 constexpr int THREADS = WARPS * 32;
-constexpr int COPIES = 8;
 constexpr unsigned long long WAIT_NS = 1000000000ull;
 
 __device__ int g_cs_error = 0;
@@ -73,8 +74,8 @@ __host__ __device__ inline size_t r16(size_t v) { return (v + 15) & ~size_t(15);
 // Shared-memory layout of a block (byte offsets, every region 16-byte aligned).
 struct Carve {
   size_t xs, yp, bar, words;
-  __host__ __device__ Carve(int E, int n_sub, int NB, int rpp) {
-    xs = r16((size_t)(E + 1) * COPIES * 16);            // slice + the null entry
+  __host__ __device__ Carve(int E, int n_sub, int NB, int rpp, int copies) {
+    xs = r16((size_t)(E + 1) * copies * 16);            // slice + the null entry
     yp = r16(xs + (size_t)n_sub * NB * 8 * 4);
     bar = r16(yp + (size_t)NB * rpp * 4);
     words = bar + 16 + WARPS * 4;                     // mbarrier, abort flag, per-warp max|x'|
@@ -93,7 +94,7 @@ struct Args {
   int words_cap;        // words the shared buffer holds (a multiple of 32)
 };
 
-template <int NB, int EPW>
+template <int NB, int EPW, int COPIES>
 __global__ void __launch_bounds__(THREADS, 1) k_gemv_cs(Args a) {
   constexpr int SLOT = EPW == 3 ? 21 : 32;
   const Layer& L = a.L;
@@ -106,7 +107,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_cs(Args a) {
   const int slice0 = p * E, E_p = max(0, min(E, L.k1 - slice0));
   const int n_sub = L.n_sub;
   const int B = a.batch;
-  const Carve cv(E, n_sub, NB, RPP);
+  const Carve cv(E, n_sub, NB, RPP, COPIES);
   uint4* cbs = reinterpret_cast<uint4*>(smem);                        // [E][8]
   float* xs = reinterpret_cast<float*>(smem + cv.xs);                 // [n_sub][NB][8]
   int* yp = reinterpret_cast<int*>(smem + cv.yp);                     // [NB][RPP] fixed point
@@ -148,7 +149,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_cs(Args a) {
     v1 = __ldg(cb + min(k1, E_p - 1));
     // the copies are written in a lane-rotated order: at every store the eight lanes of a
     // quarter-warp write eight different copies, i.e. eight different bank groups
-    const int rot = threadIdx.x & (COPIES - 1);
+    const int rot = ((threadIdx.x & 7) / (8 / COPIES)) & (COPIES - 1);
     if (k0 < E_p)
 #pragma unroll
       for (int cc = 0; cc < COPIES; ++cc) cbs[k0 * COPIES + ((cc + rot) & (COPIES - 1))] = v0;
@@ -475,12 +476,29 @@ __global__ void __launch_bounds__(256) k_cs_finalize(Layer L, const float* __res
   }
 }
 
-template <int NB, int EPW>
+template <int NB, int EPW, int COPIES>
 static cudaError_t launch_cfg(const Args& a, size_t smem, cudaStream_t s) {
-  auto k = k_gemv_cs<NB, EPW>;
+  auto k = k_gemv_cs<NB, EPW, COPIES>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(k, dim3(a.L.cs_P * a.L.cs_H), THREADS, smem, s, a);
+}
+
+}  // namespace csg
+
+// Failure-detection self-test: one thread waits on a freshly initialised mbarrier that nothing
+// will ever complete, with the same bounded try-wait loop the decode kernel uses but the
+// caller's limit.  When the limit passes it records code 7 and returns; no copy is in flight.
+namespace csg {
+__global__ void k_wait_probe(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(su32(&bar)) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    const uint64_t t0 = now_ns();
+    while (!mbar_try(su32(&bar), 0u))
+      if (now_ns() - t0 > limit_ns) { atomicExch(&g_cs_error, 7); break; }
+  }
 }
 
 }  // namespace csg
@@ -506,24 +524,43 @@ cudaError_t launch_gemv_cs(const Layer& L, const void* x, vqlin_dtype xt, int ba
   if (!ws || ws_bytes < need) return cudaSuccess;
   const int NB = batch == 1 ? 1 : (batch == 2 ? 2 : 4);
   const size_t smem_max = 227 * 1024;
-  const Carve cv(L.cs_E, L.n_sub, NB, L.cs_rpp);
+  // 8 codebook copies (conflict-free gathers) unless that forces the entry stream into
+  // several chunks while 4 copies would hold it whole
+  const int need_words = (int)((L.cs_max_words + 31) & ~31ll);
+  int copies = 8;
+  {
+    const Carve c8(L.cs_E, L.n_sub, NB, L.cs_rpp, 8), c4(L.cs_E, L.n_sub, NB, L.cs_rpp, 4);
+    if (c8.total(need_words) > smem_max && c4.total(need_words) <= smem_max) copies = 4;
+  }
+  const Carve cv(L.cs_E, L.n_sub, NB, L.cs_rpp, copies);
   if (cv.total(64) > smem_max) return cudaSuccess;
   Args a;
   a.L = L; a.x = x; a.xt = xt; a.batch = batch; a.planes = reinterpret_cast<float*>(ws);
   int cap = (int)(((smem_max - cv.words) / 10) & ~31ll);     // 8 + 2 bytes per word, whole groups of 32
-  const int need_words = (int)((L.cs_max_words + 31) & ~31ll);
   if (need_words < cap) cap = need_words;
   a.words_cap = cap < 32 ? 32 : cap;
   const size_t smem = cv.total(a.words_cap);
   cudaError_t e;
-  if (L.cs_epw == 3) {
-    if (NB == 1) e = launch_cfg<1, 3>(a, smem, s);
-    else if (NB == 2) e = launch_cfg<2, 3>(a, smem, s);
-    else e = launch_cfg<4, 3>(a, smem, s);
+  if (copies == 8) {
+    if (L.cs_epw == 3) {
+      if (NB == 1) e = launch_cfg<1, 3, 8>(a, smem, s);
+      else if (NB == 2) e = launch_cfg<2, 3, 8>(a, smem, s);
+      else e = launch_cfg<4, 3, 8>(a, smem, s);
+    } else {
+      if (NB == 1) e = launch_cfg<1, 2, 8>(a, smem, s);
+      else if (NB == 2) e = launch_cfg<2, 2, 8>(a, smem, s);
+      else e = launch_cfg<4, 2, 8>(a, smem, s);
+    }
   } else {
-    if (NB == 1) e = launch_cfg<1, 2>(a, smem, s);
-    else if (NB == 2) e = launch_cfg<2, 2>(a, smem, s);
-    else e = launch_cfg<4, 2>(a, smem, s);
+    if (L.cs_epw == 3) {
+      if (NB == 1) e = launch_cfg<1, 3, 4>(a, smem, s);
+      else if (NB == 2) e = launch_cfg<2, 3, 4>(a, smem, s);
+      else e = launch_cfg<4, 3, 4>(a, smem, s);
+    } else {
+      if (NB == 1) e = launch_cfg<1, 2, 4>(a, smem, s);
+      else if (NB == 2) e = launch_cfg<2, 2, 4>(a, smem, s);
+      else e = launch_cfg<4, 2, 4>(a, smem, s);
+    }
   }
   if (e != cudaSuccess) return e;
   const float* planes = a.planes;
@@ -538,3 +575,11 @@ cudaError_t launch_gemv_cs(const Layer& L, const void* x, vqlin_dtype xt, int ba
 }
 
 }  // namespace vqlin
+
+extern "C" vqlin_status vqlin_selftest_wait_timeout(int32_t limit_us, void* stream) {
+  using namespace vqlin;
+  if (limit_us < 1 || limit_us > 1000000) { set_error("limit_us = %d: must be 1..1000000", limit_us); return VQLIN_ERR_INVALID_ARG; }
+  note_launches(1);
+  csg::k_wait_probe<<<1, 32, 0, (cudaStream_t)stream>>>((unsigned long long)limit_us * 1000ull);
+  return cuda_status(cudaGetLastError(), "self-test launch");
+}

@@ -85,11 +85,12 @@ vqlin_last_error = _sig("vqlin_last_error", C.c_char_p, [])
 vqlin_abi_version = _sig("vqlin_abi_version", C.c_int32, [])
 vqlin_device_error = _sig("vqlin_device_error", _S, [C.POINTER(C.c_int32)])
 vqlin_kernel_launches = _sig("vqlin_kernel_launches", C.c_uint64, [])
+vqlin_selftest_wait_timeout = _sig("vqlin_selftest_wait_timeout", _S, [C.c_int32, C.c_void_p])
 
 EXPORTS = ["vqlin_create", "vqlin_destroy", "vqlin_get_info", "vqlin_dequant", "vqlin_gemv", "vqlin_gemm",
            "vqlin_gemm_workspace_size", "vqlin_unpack_indices", "vqlin_status_string", "vqlin_last_error",
            "vqlin_abi_version", "vqlin_device_error", "vqlin_gemv_ws", "vqlin_gemv_workspace_size", "vqlin_gemv_noalloc",
-           "vqlin_kernel_launches"]
+           "vqlin_kernel_launches", "vqlin_selftest_wait_timeout"]
 
 
 def device_error() -> int:
