@@ -16,9 +16,10 @@ the launching stream, with a barrier and a device synchronisation on both
 sides; the maximum over ranks is reported.  Weights rotate through enough
 independent copies to exceed 3x the L2 size, so every step streams its weights
 from HBM.  SM clocks and throttle reasons are sampled through NVML during the
-timed region.  `e2e` repeats the K steps eagerly through the same C-ABI calls
-with the step's input copied from pinned host memory and its output read back
-to pinned host memory (stream synchronised) every step.
+timed region.  `e2e` repeats the K steps through the same C-ABI calls with the
+step's input copied from pinned host memory and its output read back to pinned
+host memory every step: each step is one CUDA graph [copy x in, call(s), copy y
+out] replayed and waited for on the host (stream synchronised).
 
 One JSON line is printed by rank 0.  Under torchrun (N > 1) every rank runs an
 independent replica (the layer shards by rows with no exchange; here each rank
@@ -269,6 +270,23 @@ def run_vqlin(args, rank, world, dist):
     x_host = [torch.from_numpy(np.ascontiguousarray(wl.xs[li][:B]).view(np.int16)).pin_memory() for li, B in wl.calls]
     y_host = [torch.empty((B, wl.layers[li].n_out), dtype=torch.int16).pin_memory() for li, B in wl.calls]
     n_e2e = args.steps
+    # one CUDA graph per weight copy holding a whole step as a user runs it: the host->device
+    # copy of x from pinned memory, the C-ABI call(s), the device->host copy of y; every timed
+    # step replays one and waits for y on the host
+    n_g = min(n_copies, n_e2e)
+    e2e_graphs = []
+    for gi in range(n_g):
+        ge = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(ge, stream=stream):
+            cap = torch.cuda.current_stream().cuda_stream
+            for k in range(len(wl.calls)):
+                xs[k].view(torch.int16).copy_(x_host[k], non_blocking=True)
+            step(gi, cap)
+            for k in range(len(wl.calls)):
+                y_host[k].copy_(ys[k].view(torch.int16), non_blocking=True)
+        e2e_graphs.append(ge)
+    for ge in e2e_graphs:
+        ge.replay()
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
@@ -276,14 +294,11 @@ def run_vqlin(args, rank, world, dist):
     with torch.cuda.stream(stream):
         f0.record(stream)
         for i in range(n_e2e):
-            for k in range(len(wl.calls)):
-                xs[k].view(torch.int16).copy_(x_host[k], non_blocking=True)
-            step(i, s_ptr)
-            for k in range(len(wl.calls)):
-                y_host[k].copy_(ys[k].view(torch.int16), non_blocking=True)
+            e2e_graphs[i % n_g].replay()
             stream.synchronize()
         f1.record(stream)
     torch.cuda.synchronize()
+    del e2e_graphs
     e2e_ms = f0.elapsed_time(f1)
     if dist:
         t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
