@@ -789,8 +789,9 @@ cudaError_t launch_gemv_tc(const Layer& L, const void* x, vqlin_dtype xt, int ba
   const int n_rg = (n_rt + a.rtt - 1) / a.rtt;
   // ---- warp-task kernel: needs an fp32 accumulator (y itself, or the caller's workspace)
   //      and x' for every column next to the codebooks.  When one block task already
-  //      covers every column, the block-task kernel below writes y in a single grid.
-  if (a.n_chunks > 1) {
+  //      covers every column and the tasks fit in one wave (the block-task kernel runs one
+  //      block per SM), the block-task kernel below writes y in a single grid.
+  if (a.n_chunks > 1 || n_rg > sms) {
     float* acc = nullptr;
     if (yt == VQLIN_F32) acc = reinterpret_cast<float*>(y);
     else if (ws && ws_bytes >= gemv_workspace_bytes(L, batch)) acc = reinterpret_cast<float*>(ws);
