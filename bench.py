@@ -96,6 +96,12 @@ def make_workload(name: str, batch: int) -> Workload:
         L, Xb = synth.prefill(2048)
         return Workload("prefill_2048x4096x4096_d8_k65536", [L], [Xb], [(0, 2048)], "gemm",
                         "X 2048x4096 bf16 times the q_proj-shaped VQ weight, bf16 Y")
+    if name.startswith("vlen"):
+        d = int(name[4:])
+        L, xb = synth.vlen(d, batch)
+        return Workload("vlen_4096x4096_d%d_k4096_b%d" % (d, batch), [L], [xb], [(0, batch)], "gemv",
+                        "4096x4096, d=%d, K=4096 fp16 codebook (12-bit codes, %.3g bits/weight), fp16 row+col "
+                        "scales, 1%% CSR outliers, fp16 x/y, batch %d" % (d, 12.0 / d, batch))
     raise SystemExit("unknown config " + name)
 
 
@@ -415,7 +421,8 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="vqlin", choices=["vqlin", "reference"])
-    ap.add_argument("--config", default="qproj", choices=["qproj", "tiny", "downproj", "smollm", "prefill"])
+    ap.add_argument("--config", default="qproj",
+                    choices=["qproj", "tiny", "downproj", "smollm", "prefill", "vlen4", "vlen6", "vlen8", "vlen12"])
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

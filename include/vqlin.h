@@ -85,7 +85,7 @@ extern "C" {
 typedef enum {
   VQLIN_OK = 0,
   VQLIN_ERR_INVALID_ARG = 1,  /* NULL pointer, bad size, bad stride or alignment   */
-  VQLIN_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. d not in {4,8})    */
+  VQLIN_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. d not in {4,6,8,12}) */
   VQLIN_ERR_INVALID_DATA = 3, /* index >= k, malformed CSR, non-finite value        */
   VQLIN_ERR_OOM = 4,          /* device or host allocation failed                   */
   VQLIN_ERR_CUDA = 5,         /* a CUDA call or kernel launch failed                */
@@ -103,7 +103,9 @@ typedef struct vqlin_handle vqlin_handle;
  */
 typedef struct {
   int32_t n_out, n_in;        /* W is n_out x n_in; both >= 1                         */
-  int32_t d;                  /* sub-vector length; kernels support 4 and 8            */
+  int32_t d;                  /* sub-vector length: 4, 6, 8 or 12 (VPTQ's vector
+                                 lengths); the tensor-core and codebook-stationary
+                                 decode paths are d = 8, the others run CUDA cores    */
   int32_t src_on_host;        /* 0: pointers below are device pointers; 1: host        */
 
   /* main body */

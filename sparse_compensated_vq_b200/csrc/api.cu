@@ -147,7 +147,10 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
   // ---- shape checks
   if (D->n_out < 1 || D->n_in < 1) { set_error("n_out and n_in must be >= 1"); return VQLIN_ERR_INVALID_ARG; }
   if (D->d < 1 || D->d > 64) { set_error("d = %d out of range", D->d); return VQLIN_ERR_INVALID_ARG; }
-  if (D->d != 4 && D->d != 8) { set_error("d = %d: kernels support d in {4, 8}", D->d); return VQLIN_ERR_UNSUPPORTED; }
+  if (D->d != 4 && D->d != 6 && D->d != 8 && D->d != 12) {
+    set_error("d = %d: kernels support d in {4, 6, 8, 12}", D->d);
+    return VQLIN_ERR_UNSUPPORTED;
+  }
   if (D->bits1 < 1 || D->bits1 > 16 || D->k1 < 1 || (int64_t)D->k1 > (1ll << D->bits1)) {
     set_error("need 1 <= bits1 <= 16 and 1 <= k1 <= 2^bits1 (k1 = %d, bits1 = %d)", D->k1, D->bits1);
     return VQLIN_ERR_INVALID_ARG;

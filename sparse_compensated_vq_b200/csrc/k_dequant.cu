@@ -69,14 +69,23 @@ __global__ void __launch_bounds__(256) k_dequant_body(Layer L, __half* __restric
         if (e2) S = S + (double)__half2float(e2[k]);
         outv[k] = exact_f16(S, L.rs, L.cs, i, j);
       }
-      if (!L.colmap && q0 + D <= L.n_main && (((reinterpret_cast<uintptr_t>(Wrow + q0)) & (2 * D - 1)) == 0)) {
-        if (D == 8) {
-          uint4 v = make_uint4(outv[0] | (uint32_t(outv[1]) << 16), outv[2] | (uint32_t(outv[3]) << 16),
-                               outv[4] | (uint32_t(outv[5]) << 16), outv[6] | (uint32_t(outv[7]) << 16));
-          *reinterpret_cast<uint4*>(Wrow + q0) = v;
+      // vector stores of the D outputs: 16-byte units for D = 8, 8-byte for D = 4 and 12,
+      // 4-byte for D = 6, when the destination is aligned to that unit
+      constexpr int VB = D % 8 == 0 ? 16 : (D % 4 == 0 ? 8 : 4);
+      if (!L.colmap && q0 + D <= L.n_main && (((reinterpret_cast<uintptr_t>(Wrow + q0)) & (VB - 1)) == 0)) {
+        uint32_t pk[D / 2];
+#pragma unroll
+        for (int k = 0; k < D / 2; ++k) pk[k] = outv[2 * k] | (uint32_t(outv[2 * k + 1]) << 16);
+        if constexpr (VB == 16) {
+#pragma unroll
+          for (int i = 0; i < D / 8; ++i)
+            reinterpret_cast<uint4*>(Wrow + q0)[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        } else if constexpr (VB == 8) {
+#pragma unroll
+          for (int i = 0; i < D / 4; ++i) reinterpret_cast<uint2*>(Wrow + q0)[i] = make_uint2(pk[2 * i], pk[2 * i + 1]);
         } else {
-          uint2 v = make_uint2(outv[0] | (uint32_t(outv[1]) << 16), outv[2] | (uint32_t(outv[3]) << 16));
-          *reinterpret_cast<uint2*>(Wrow + q0) = v;
+#pragma unroll
+          for (int i = 0; i < D / 2; ++i) reinterpret_cast<uint32_t*>(Wrow + q0)[i] = pk[i];
         }
       } else {
 #pragma unroll
@@ -250,8 +259,12 @@ cudaError_t launch_dequant(const Layer& L, __half* W, int64_t ldw, cudaStream_t 
   }
   if (work > 0) {
     note_launches(1);
-    if (L.d == 8) k_dequant_body<8><<<grid_for(work, 256), 256, 0, s>>>(L, W, ldw);
-    else k_dequant_body<4><<<grid_for(work, 256), 256, 0, s>>>(L, W, ldw);
+    switch (L.d) {
+      case 8: k_dequant_body<8><<<grid_for(work, 256), 256, 0, s>>>(L, W, ldw); break;
+      case 4: k_dequant_body<4><<<grid_for(work, 256), 256, 0, s>>>(L, W, ldw); break;
+      case 6: k_dequant_body<6><<<grid_for(work, 256), 256, 0, s>>>(L, W, ldw); break;
+      default: k_dequant_body<12><<<grid_for(work, 256), 256, 0, s>>>(L, W, ldw); break;
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

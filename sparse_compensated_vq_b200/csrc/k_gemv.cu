@@ -20,34 +20,46 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-template <int D>
-__device__ __forceinline__ void load_centroid(const __half* base, uint32_t idx, float* c) {
-  if (D == 8) {
-    uint4 u = __ldg(reinterpret_cast<const uint4*>(base) + idx);
-    const __half2* h = reinterpret_cast<const __half2*>(&u);
+// One centroid of D fp16 elements (D in {4, 6, 8, 12}) as floats, with the widest vector
+// loads the entry alignment allows: D*2 bytes per entry, so 16-byte loads for D = 8, 8-byte
+// loads for D = 4 and 12, 4-byte loads for D = 6.
+template <int D, bool SMEM>
+__device__ __forceinline__ void load_centroid_any(const __half* base, uint32_t idx, float* c) {
+  uint32_t w[D / 2];
+  if constexpr (D % 8 == 0) {
+    const uint4* p = reinterpret_cast<const uint4*>(base + (size_t)idx * D);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) { float2 f = __half22float2(h[k]); c[2 * k] = f.x; c[2 * k + 1] = f.y; }
+    for (int i = 0; i < D / 8; ++i) {
+      const uint4 u = SMEM ? p[i] : __ldg(p + i);
+      w[4 * i] = u.x; w[4 * i + 1] = u.y; w[4 * i + 2] = u.z; w[4 * i + 3] = u.w;
+    }
+  } else if constexpr (D % 4 == 0) {
+    const uint2* p = reinterpret_cast<const uint2*>(base + (size_t)idx * D);
+#pragma unroll
+    for (int i = 0; i < D / 4; ++i) {
+      const uint2 u = SMEM ? p[i] : __ldg(p + i);
+      w[2 * i] = u.x; w[2 * i + 1] = u.y;
+    }
   } else {
-    uint2 u = __ldg(reinterpret_cast<const uint2*>(base) + idx);
-    const __half2* h = reinterpret_cast<const __half2*>(&u);
+    const uint32_t* p = reinterpret_cast<const uint32_t*>(base + (size_t)idx * D);
 #pragma unroll
-    for (int k = 0; k < 2; ++k) { float2 f = __half22float2(h[k]); c[2 * k] = f.x; c[2 * k + 1] = f.y; }
+    for (int i = 0; i < D / 2; ++i) w[i] = SMEM ? p[i] : __ldg(p + i);
+  }
+#pragma unroll
+  for (int k = 0; k < D / 2; ++k) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+    c[2 * k] = f.x; c[2 * k + 1] = f.y;
   }
 }
 
 template <int D>
+__device__ __forceinline__ void load_centroid(const __half* base, uint32_t idx, float* c) {
+  load_centroid_any<D, false>(base, idx, c);
+}
+
+template <int D>
 __device__ __forceinline__ void load_centroid_smem(const __half* base, uint32_t idx, float* c) {
-  if (D == 8) {
-    uint4 u = reinterpret_cast<const uint4*>(base)[idx];
-    const __half2* h = reinterpret_cast<const __half2*>(&u);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) { float2 f = __half22float2(h[k]); c[2 * k] = f.x; c[2 * k + 1] = f.y; }
-  } else {
-    uint2 u = reinterpret_cast<const uint2*>(base)[idx];
-    const __half2* h = reinterpret_cast<const __half2*>(&u);
-#pragma unroll
-    for (int k = 0; k < 2; ++k) { float2 f = __half22float2(h[k]); c[2 * k] = f.x; c[2 * k + 1] = f.y; }
-  }
+  load_centroid_any<D, true>(base, idx, c);
 }
 
 constexpr int kThreads = 256;
@@ -55,7 +67,7 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kRPW = 2;                 // rows per warp
 constexpr int kRowsPerCta = kWarps * kRPW;
 
-// Generic kernel: any field width <= 32, d in {4, 8}, residual and outlier
+// Generic kernel: any field width <= 32, d in {4, 6, 8, 12}, residual and outlier
 // blocks, batch <= NB.  x' is staged through shared memory in column chunks.
 template <int D, int NB, bool CB_SMEM>
 __global__ void __launch_bounds__(kThreads) k_gemv_generic(Layer L, const void* __restrict__ x, vqlin_dtype xt,
@@ -70,16 +82,16 @@ __global__ void __launch_bounds__(kThreads) k_gemv_generic(Layer L, const void* 
   const __half* cb2 = L.cb2;
   const __half* cbo = L.cbo;
   if (CB_SMEM) {
-    const int n16 = ((L.k1 + L.k2 + L.ko) * D * 2) / 16;   // all three are whole multiples of 8 bytes
+    const int n16 = ((L.k1 + L.k2 + L.ko) * D * 2) / 16;   // all three are whole multiples of 4 bytes
     const uint4* srcs[3] = {reinterpret_cast<const uint4*>(L.cb1), reinterpret_cast<const uint4*>(L.cb2),
                             reinterpret_cast<const uint4*>(L.cbo)};
     int lens[3] = {L.k1 * D * 2, L.k2 * D * 2, L.ko * D * 2};
     unsigned char* dst = reinterpret_cast<unsigned char*>(cb1s);
     for (int part = 0; part < 3; ++part) {
-      // copy in 8-byte units (d = 4 entries are 8 bytes)
-      const uint2* s2 = reinterpret_cast<const uint2*>(srcs[part]);
-      uint2* d2 = reinterpret_cast<uint2*>(dst);
-      for (int t = threadIdx.x; t < lens[part] / 8; t += kThreads) d2[t] = __ldg(s2 + t);
+      // copy in 4-byte units (an entry is 2*d bytes, d even)
+      const uint32_t* s4 = reinterpret_cast<const uint32_t*>(srcs[part]);
+      uint32_t* d4 = reinterpret_cast<uint32_t*>(dst);
+      for (int t = threadIdx.x; t < lens[part] / 4; t += kThreads) d4[t] = __ldg(s4 + t);
       dst += lens[part];
     }
     (void)n16;
@@ -231,7 +243,12 @@ static cudaError_t launch_generic(const Layer& L, const void* x, vqlin_dtype xt,
 
 cudaError_t launch_gemv_generic(const Layer& L, const void* x, vqlin_dtype xt, int batch, void* y, vqlin_dtype yt,
                                 cudaStream_t s) {
-  return L.d == 8 ? launch_generic<8>(L, x, xt, batch, y, yt, s) : launch_generic<4>(L, x, xt, batch, y, yt, s);
+  switch (L.d) {
+    case 8: return launch_generic<8>(L, x, xt, batch, y, yt, s);
+    case 4: return launch_generic<4>(L, x, xt, batch, y, yt, s);
+    case 6: return launch_generic<6>(L, x, xt, batch, y, yt, s);
+    default: return launch_generic<12>(L, x, xt, batch, y, yt, s);
+  }
 }
 
 cudaError_t launch_gemv(const Layer& L, const void* x, vqlin_dtype xt, int batch, void* y, vqlin_dtype yt,

@@ -17,6 +17,9 @@ SmolLM2-1.7B layers at 2-4 bits per weight; seeds PCG64(20260000 + n)):
   3 smollm    the seven linears of a SmolLM2-1.7B decoder layer, d=8, K=256,
               2% outliers placed with column probability ~ |z|^4, z ~ N(0,1)
   4 prefill   X 2048x4096 bf16 times the qproj-shaped weight
+  5 vlen      4096x4096 at vector length d in {4, 6, 8, 12} with a K=4096 fp16 codebook
+              (12-bit codes: 3, 2, 1.5, 1 bits/weight), row+col scales, 1% uniform
+              outliers: VPTQ's vector-length trend (one seed per d)
 """
 from __future__ import annotations
 
@@ -285,3 +288,10 @@ def prefill(m: int = 2048):
     L = random_layer(rng, 4096, 4096, 8, 65536, 16, cb_std=0.02, row_scale=True, col_scale=True,
                      outlier_frac=0.01, outlier_scale=0.1, name="prefill_qproj_4096x4096_d8_k65536")
     return L, activations(rng, m, 4096, "bf16")
+
+
+def vlen(d: int, batch: int = 1):
+    rng = rng_for(5 * 100 + d)
+    L = random_layer(rng, 4096, 4096, d, 4096, 12, cb_std=0.02, row_scale=True, col_scale=True,
+                     outlier_frac=0.01, outlier_scale=0.1, name="vlen_4096x4096_d%d_k4096" % d)
+    return L, activations(rng, batch, 4096, "f16")

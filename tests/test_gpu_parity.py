@@ -40,6 +40,11 @@ def small_layers():
         dict(n_out=50, n_in=64, d=8, k1=8192, bits1=13, nnz=0, n_ocols=5, ko=8192, bits_o=13),
         dict(n_out=9, n_in=40, d=8, k1=65536, bits1=16, k2=65536, bits2=16, nnz=20),
         dict(n_out=300, n_in=24, d=4, k1=3, bits1=2, row_scale=False, nnz=100),
+        # VPTQ's other vector lengths (CUDA-core decode path)
+        dict(n_out=45, n_in=130, d=6, k1=256, bits1=8, col_scale=True, nnz=80),
+        dict(n_out=70, n_in=300, d=12, k1=4096, bits1=12, k2=256, bits2=8, nnz=90, n_ocols=10, ko=64, bits_o=6),
+        dict(n_out=19, n_in=96, d=6, k1=1, bits1=1, nnz=5),
+        dict(n_out=40, n_in=192, d=12, k1=512, bits1=9, col_scale=True, nnz=30),
     ]
     out = []
     for t, kw in enumerate(specs):
@@ -261,7 +266,7 @@ def run_gemm(vq, L, Xbits, xdt, ydt):
     return G.to_f64(Y)
 
 
-@pytest.mark.parametrize("t", [0, 1, 4])
+@pytest.mark.parametrize("t", [0, 1, 4, 10, 11])
 @pytest.mark.parametrize("M", [1, 77, 256])
 def test_gemm_small(vq, t, M):
     L = SMALL[t]

@@ -170,6 +170,11 @@ CASES = [
     dict(n_out=4, n_in=19, d=4, k1=16, bits1=4, n_ocols=5, ko=9, bits_o=4, col_scale=True, nnz=6),  # outlier block
     dict(n_out=3, n_in=26, d=8, k1=4096, bits1=12, k2=4096, bits2=12, n_ocols=3, ko=256, bits_o=8, nnz=10),
     dict(n_out=2, n_in=12, d=4, k1=65536, bits1=16, col_scale=True, row_scale=False, nnz=0),
+    # VPTQ's other vector lengths
+    dict(n_out=4, n_in=17, d=6, k1=9, bits1=4, col_scale=True, nnz=5),                      # d = 6, ragged tail
+    dict(n_out=3, n_in=30, d=6, k1=16, bits1=4, k2=5, bits2=3, n_ocols=7, ko=3, bits_o=2, nnz=4),
+    dict(n_out=3, n_in=29, d=12, k1=32, bits1=5, col_scale=True, nnz=6),                    # d = 12, ragged tail
+    dict(n_out=2, n_in=40, d=12, k1=256, bits1=8, k2=16, bits2=4, n_ocols=13, ko=7, bits_o=3, col_scale=True, nnz=5),
 ]
 
 
@@ -244,12 +249,13 @@ def test_rvq_decodes_all_k1_times_k2_pairs():
     assert (oracle.dequant_exact(L0) == oracle.dequant_exact(single)).all()
 
 
-def test_one_hot_codebook_gather_sum():
+@pytest.mark.parametrize("d", [4, 6, 8, 12])
+def test_one_hot_codebook_gather_sum(d):
     # C[k] = e_(k mod d): y_i = r_i * sum_s c_j x_j with j = s*d + (idx mod d)
-    rng = np.random.default_rng(12)
-    d, k = 8, 64
+    rng = np.random.default_rng(12 + d)
+    k = 64
     cb = np.zeros((k, d)); cb[np.arange(k), np.arange(k) % d] = 1.0
-    n_out, n_in = 7, 40
+    n_out, n_in = 7, 5 * d
     fields = rng.integers(0, k, size=(n_out, n_in // d)).astype(np.uint32)
     rs = synth.f16_bits(rng.uniform(0.5, 1.5, n_out)); cs = synth.f16_bits(rng.uniform(0.5, 1.5, n_in))
     L = synth.LayerData(n_out=n_out, n_in=n_in, d=d, k1=k, bits1=6, codes=synth.pack_fields(fields, 6),
