@@ -133,23 +133,33 @@ __global__ void __launch_bounds__(kThreads) k_gemv_generic(Layer L, const void* 
       const int row = row0 + r;
       if (row >= L.n_out) break;
       const uint8_t* rowp = L.codes + (int64_t)row * L.stride;
-      for (int s = s0 + lane; s < s1; s += 32) {
-        uint32_t f = read_field(rowp, s, L.w);
-        float c[D];
-        if (CB_SMEM) load_centroid_smem<D>(cb1, f & m1, c); else load_centroid<D>(cb1, f & m1, c);
-        if (cb2) {
-          float c2[D];
-          if (CB_SMEM) load_centroid_smem<D>(cb2, f >> L.bits1, c2); else load_centroid<D>(cb2, f >> L.bits1, c2);
+      // four sub-vectors per lane and round: their fields are read (clamped) before any use
+      constexpr int UF = 4;
+      for (int sb = s0 + lane; sb < s1; sb += 32 * UF) {
+        uint32_t fs[UF];
 #pragma unroll
-          for (int k = 0; k < D; ++k) c[k] += c2[k];
-        }
-        const float* xv = xs + (s - s0) * D;
+        for (int u = 0; u < UF; ++u) fs[u] = read_field(rowp, min(sb + 32 * u, s1 - 1), L.w);
 #pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          float a = acc[r][b];
+        for (int u = 0; u < UF; ++u) {
+          const int s = sb + 32 * u;
+          if (s >= s1) break;
+          const uint32_t f = fs[u];
+          float c[D];
+          if (CB_SMEM) load_centroid_smem<D>(cb1, f & m1, c); else load_centroid<D>(cb1, f & m1, c);
+          if (cb2) {
+            float c2[D];
+            if (CB_SMEM) load_centroid_smem<D>(cb2, f >> L.bits1, c2); else load_centroid<D>(cb2, f >> L.bits1, c2);
 #pragma unroll
-          for (int k = 0; k < D; ++k) a = fmaf(c[k], xv[b * chunk + k], a);
-          acc[r][b] = a;
+            for (int k = 0; k < D; ++k) c[k] += c2[k];
+          }
+          const float* xv = xs + (s - s0) * D;
+#pragma unroll
+          for (int b = 0; b < NB; ++b) {
+            float a = acc[r][b];
+#pragma unroll
+            for (int k = 0; k < D; ++k) a = fmaf(c[k], xv[b * chunk + k], a);
+            acc[r][b] = a;
+          }
         }
       }
     }
