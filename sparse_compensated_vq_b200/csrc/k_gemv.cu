@@ -88,10 +88,18 @@ __global__ void __launch_bounds__(kThreads) k_gemv_generic(Layer L, const void* 
     int lens[3] = {L.k1 * D * 2, L.k2 * D * 2, L.ko * D * 2};
     unsigned char* dst = reinterpret_cast<unsigned char*>(cb1s);
     for (int part = 0; part < 3; ++part) {
-      // copy in 4-byte units (an entry is 2*d bytes, d even)
+      // copy in 4-byte units (an entry is 2*d bytes, d even), eight loads in flight per thread
       const uint32_t* s4 = reinterpret_cast<const uint32_t*>(srcs[part]);
       uint32_t* d4 = reinterpret_cast<uint32_t*>(dst);
-      for (int t = threadIdx.x; t < lens[part] / 4; t += kThreads) d4[t] = __ldg(s4 + t);
+      const int n4 = lens[part] / 4;
+      for (int t0 = threadIdx.x; t0 < n4; t0 += 8 * kThreads) {
+        uint32_t v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = __ldg(s4 + min(t0 + u * kThreads, n4 - 1));
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (t0 + u * kThreads < n4) d4[t0 + u * kThreads] = v[u];
+      }
       dst += lens[part];
     }
     (void)n16;
@@ -193,15 +201,7 @@ __global__ void __launch_bounds__(kThreads) k_gemv_generic(Layer L, const void* 
     float sp[NB];
 #pragma unroll
     for (int b = 0; b < NB; ++b) sp[b] = 0.f;
-    if (L.nnz > 0) {
-      for (int e = L.row_ptr[row] + lane; e < L.row_ptr[row + 1]; e += 32) {
-        const float dl = L.delta[e];
-        const int j = L.col[e];
-#pragma unroll
-        for (int b = 0; b < NB; ++b)
-          if (b < batch) sp[b] = fmaf(dl, load_as_float(x, xt, (int64_t)b * L.n_in + j), sp[b]);
-      }
-    }
+    if (L.nnz > 0) sparse_row_terms<NB>(L, x, xt, batch, row, lane, 32, sp);
     const float rsc = L.rs ? __half2float(L.rs[row]) : 1.f;
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
