@@ -14,5 +14,6 @@ from .oracle import (  # noqa: F401
     dequant_f64,
     gemv_f64,
     vptq_compression_ratio,
+    assign_f32,
     OracleError,
 )

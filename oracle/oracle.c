@@ -336,3 +336,49 @@ double oracle_vptq_compression_ratio(int64_t n_elems, int32_t V, int64_t k) {
   double index = (double)n_elems * (double)bits / (double)V;
   return original / (codebook + index);
 }
+
+/* ---------------------------------------------------------------- nearest-centroid assignment
+   VPTQ page, "Step 3: Vector quantization of column n": Q_V(v) = argmin_i ||v - C_i||^2 (plain
+   Euclidean distance), and "Residual Vector Quantization": i1 = Q_1(v), v_res = v - C[i1],
+   i2 = argmin_j ||v_res - Cres_j||^2.  The pages fix no precision; this restates the decision
+   in the library kernel's precision so both sides take it identically: every difference,
+   square and running sum is one IEEE binary32 operation rounded to nearest (no fused
+   multiply-add; built with -ffp-contract=off), elements in order 0..d-1, centroids scanned
+   from index 0 up, and a centroid replaces the best one only when strictly closer (ties
+   keep the lowest index).  v_res is the binary32 difference v - C[i1].  fp16 inputs convert
+   to binary32 exactly. */
+static float f16_to_f32(uint16_t h) { return (float)oracle_f16_to_f64(h); }
+
+static uint32_t nearest_f32(const float* v, int32_t d, const uint16_t* C, int32_t k) {
+  uint32_t best = 0;
+  float best_d = 0.0f;
+  for (int32_t i = 0; i < k; ++i) {
+    float acc = 0.0f;
+    for (int32_t t = 0; t < d; ++t) {
+      volatile float diff = v[t] - f16_to_f32(C[(int64_t)i * d + t]);
+      volatile float sq = diff * diff;
+      acc = acc + sq;
+    }
+    if (i == 0 || acc < best_d) { best = (uint32_t)i; best_d = acc; }
+  }
+  return best;
+}
+
+int oracle_assign_f32(const uint16_t* V, int64_t n, int32_t d, const uint16_t* C1, int32_t k1,
+                      const uint16_t* C2, int32_t k2, uint32_t* idx1, uint32_t* idx2) {
+  float v[64];
+  if (d < 1 || d > 64 || k1 < 1 || (k2 > 0 && !C2)) return ORACLE_BAD_VALUE;
+  for (int64_t e = 0; e < n * d; ++e) if (((V[e] >> 10) & 0x1F) == 31) return ORACLE_BAD_VALUE;
+  for (int64_t e = 0; e < (int64_t)k1 * d; ++e) if (((C1[e] >> 10) & 0x1F) == 31) return ORACLE_BAD_VALUE;
+  for (int64_t e = 0; e < (int64_t)k2 * d; ++e) if (((C2[e] >> 10) & 0x1F) == 31) return ORACLE_BAD_VALUE;
+  for (int64_t s = 0; s < n; ++s) {
+    for (int32_t t = 0; t < d; ++t) v[t] = f16_to_f32(V[s * d + t]);
+    const uint32_t i1 = nearest_f32(v, d, C1, k1);
+    idx1[s] = i1;
+    if (k2 > 0) {
+      for (int32_t t = 0; t < d; ++t) { volatile float r = v[t] - f16_to_f32(C1[(int64_t)i1 * d + t]); v[t] = r; }
+      idx2[s] = nearest_f32(v, d, C2, k2);
+    }
+  }
+  return ORACLE_OK;
+}

@@ -78,6 +78,8 @@ def _load():
             lib.oracle_gemv_f64_rows.argtypes = [C.POINTER(_Layer), P, C.c_int32, P, C.c_int64, P]
             lib.oracle_vptq_compression_ratio.restype = C.c_double
             lib.oracle_vptq_compression_ratio.argtypes = [C.c_int64, C.c_int32, C.c_int64]
+            lib.oracle_assign_f32.restype = C.c_int
+            lib.oracle_assign_f32.argtypes = [P, C.c_int64, C.c_int32, P, C.c_int32, P, C.c_int32, P, P]
             _lib = lib
     return _lib
 
@@ -204,3 +206,28 @@ def gemv_f64(layer, x: np.ndarray, rows=None) -> np.ndarray:
 
 def vptq_compression_ratio(n_elems: int, V: int, k: int) -> float:
     return float(_load().oracle_vptq_compression_ratio(int(n_elems), int(V), int(k)))
+
+
+def assign_f32(V: np.ndarray, C1: np.ndarray, C2: np.ndarray | None = None):
+    """Nearest-centroid indices of fp16 sub-vectors V [n, d] (uint16 bits) in C1 [k1, d] and,
+    with a residual codebook C2 [k2, d], of v - C1[i1] in C2 (oracle.c: oracle_assign_f32).
+    Returns (idx1, idx2) as uint32 arrays; idx2 is None without C2."""
+    lib = _load()
+    V = _c(V, np.uint16)
+    C1 = _c(C1, np.uint16)
+    n, d = V.shape
+    k1 = C1.shape[0]
+    assert C1.shape[1] == d
+    i1 = np.zeros(n, np.uint32)
+    i2 = None
+    k2 = 0
+    c2p = None
+    if C2 is not None:
+        C2 = _c(C2, np.uint16)
+        assert C2.shape[1] == d
+        k2 = C2.shape[0]
+        i2 = np.zeros(n, np.uint32)
+        c2p = _ptr(C2)
+    _check(lib.oracle_assign_f32(_ptr(V), C.c_int64(n), C.c_int32(d), _ptr(C1), C.c_int32(k1), c2p, C.c_int32(k2),
+                                 _ptr(i1), _ptr(i2) if i2 is not None else None))
+    return i1, i2

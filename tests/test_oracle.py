@@ -332,3 +332,70 @@ def test_malformed_csr_is_reported():
     L.values = synth.f16_bits([1.0, 2.0, 3.0])
     with pytest.raises(oracle.OracleError):
         oracle.dequant_exact(L)
+
+
+# ---------------------------------------------------------------- nearest-centroid assignment
+# VPTQ page, "Step 3": Q_V(v) = argmin_i ||v - C_i||^2; "Residual Vector Quantization":
+# i2 = argmin_j ||(v - C1[i1]) - Cres_j||^2.  The oracle takes the decision in binary32; these
+# pins hold it to the exact (rational) argmin wherever binary32 cannot change the answer.
+U32 = 2.0 ** -24
+
+
+def _exact_sqdist(v_bits, c_bits):
+    return sum(((exact.f16_frac(int(a)) - exact.f16_frac(int(b))) ** 2 for a, b in zip(v_bits, c_bits)), Fraction(0))
+
+
+@pytest.mark.parametrize("d", [4, 6, 8, 12])
+def test_assign_matches_exact_argmin_where_binary32_cannot_decide_otherwise(d):
+    rng = np.random.default_rng(300 + d)
+    k, n = 37, 25
+    C = synth.f16_bits(rng.normal(0, 1, (k, d)))
+    V = synth.f16_bits(rng.normal(0, 1, (n, d)))
+    i1, _ = oracle.assign_f32(V, C)
+    tol = Fraction(2 * (d + 3)) * Fraction(U32)           # relative error of one binary32 distance
+    for s in range(n):
+        dist = [_exact_sqdist(V[s], C[i]) for i in range(k)]
+        best = min(dist)
+        assert dist[int(i1[s])] <= best * (1 + 2 * tol)    # the pick is (near-)optimal
+        order = sorted(range(k), key=lambda i: (dist[i], i))
+        if dist[order[1]] > best * (1 + 2 * tol):          # unique beyond rounding: must match
+            assert int(i1[s]) == order[0]
+
+
+def test_assign_exact_hits_and_ties_take_the_lowest_index():
+    rng = np.random.default_rng(41)
+    d = 8
+    base = synth.f16_bits(rng.normal(0, 1, (10, d)))
+    C = np.concatenate([base, base[[3, 7]], base]).astype(np.uint16)   # duplicates at 10, 11 and 12..21
+    V = base[[3, 7, 0, 9]]
+    i1, _ = oracle.assign_f32(V, C)
+    assert i1.tolist() == [3, 7, 0, 9]
+    # equidistant centroids: v halfway (exactly) between two candidates
+    C2 = synth.f16_bits(np.array([[0, 0, 0, 0], [2, 0, 0, 0], [1, 0, 0, 1.5], [1, 0, 0, -1.5]]))
+    V2 = synth.f16_bits(np.array([[1, 0, 0, 0]]))
+    assert oracle.assign_f32(V2, C2)[0].tolist() == [0]
+
+
+def test_residual_stage_recovers_constructed_pairs():
+    # C1 entries far apart (multiples of 8), residual entries small (multiples of 1/4, |.| <= 1):
+    # every v = C1[a] + C2[b] is exact in fp16 and its two-stage argmin is (a, b)
+    rng = np.random.default_rng(42)
+    d, k1, k2 = 6, 12, 9
+    C1 = synth.f16_bits(8.0 * rng.integers(-6, 7, (k1, d)))
+    C1 = np.unique(C1, axis=0)[:k1]
+    k1 = len(C1)
+    C2 = synth.f16_bits(0.25 * rng.integers(-4, 5, (k2, d)))
+    C2 = np.unique(C2, axis=0)
+    k2 = len(C2)
+    pairs = [(a, b) for a in range(k1) for b in range(k2)]
+    f = lambda h: h.view(np.float16).astype(np.float64)
+    V = synth.f16_bits(np.array([f(C1[a]) + f(C2[b]) for a, b in pairs]))
+    i1, i2 = oracle.assign_f32(V, C1, C2)
+    assert list(zip(i1.tolist(), i2.tolist())) == pairs
+
+
+def test_assign_rejects_non_finite_input():
+    C = synth.f16_bits(np.ones((2, 4)))
+    V = np.array([[0x7C00, 0, 0, 0]], dtype=np.uint16)     # +inf
+    with pytest.raises(oracle.OracleError):
+        oracle.assign_f32(V, C)

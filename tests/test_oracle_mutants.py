@@ -27,6 +27,11 @@ MUTANTS = {
     "outlier_codebook": ("*e1 = L->cbo + (int64_t)io * d + (p % d);",
                          "*e1 = L->cb1 + (int64_t)(io % L->k1) * d + (p % d);"),
     "col_scale_dropped": ("if (L->cs) v = v * oracle_f16_to_f64(L->cs[j]);", ";"),
+    "assign_ties_highest": ("if (i == 0 || acc < best_d) {", "if (i == 0 || acc <= best_d) {"),
+    "assign_residual_dropped": ("volatile float r = v[t] - f16_to_f32(C1[(int64_t)i1 * d + t]); v[t] = r;",
+                                "volatile float r = v[t]; v[t] = r;"),
+    "assign_element_skewed": ("volatile float diff = v[t] - f16_to_f32(C[(int64_t)i * d + t]);",
+                              "volatile float diff = v[t] - f16_to_f32(C[(int64_t)i * d + (t + 1) % d]);"),
 }
 
 
