@@ -415,6 +415,84 @@ def run_reference(args, rank, world):
 
 
 # --------------------------------------------------------------------------- main
+def run_encode(args, rank, world, dist):
+    """Nearest-centroid assignment of every sub-vector of a 4096x4096 fp16 weight (d = 8, about
+    2.1 M sub-vectors) against a K = 4096 codebook (VPTQ's Q_V).  Same timing protocol as the
+    decode bench; the roofline is the CUDA-core ALU: 3d + 1 binary32 operations per
+    (sub-vector, centroid) against 148 SMs x 128 FP32 lanes x the sampled SM clock."""
+    import torch
+    from sparse_compensated_vq_b200 import vqlin
+
+    dev = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(dev)
+    d, k, n_out, n_in = 8, 4096, 4096, 4096
+    rng = synth.rng_for(6)
+    C1 = synth.f16_bits(rng.normal(0.0, 0.02, (k, d)))
+    V = synth.f16_bits(rng.normal(0.0, 0.02, (n_out * n_in // d, d)))
+    n = V.shape[0]
+    dv = torch.from_numpy(V.view(np.int16)).cuda()
+    dc = torch.from_numpy(C1.view(np.int16)).cuda()
+    idx = torch.empty(n, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.Stream()
+
+    def step(s_ptr):
+        st = vqlin.vqlin_assign(dv.data_ptr(), n, d, dc.data_ptr(), k, None, 0, idx.data_ptr(), None, s_ptr)
+        if st != 0:
+            raise vqlin.VQLinError(st, "assign")
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step(stream.cuda_stream)
+    torch.cuda.synchronize()
+    steps = min(args.steps, 50)                   # a step is ~6 ms of ALU work
+    g = torch.cuda.CUDAGraph()
+    n0 = vqlin.vqlin_kernel_launches()
+    with torch.cuda.graph(g, stream=stream):
+        cap = torch.cuda.current_stream().cuda_stream
+        for _ in range(steps):
+            step(cap)
+    launches = vqlin.vqlin_kernel_launches() - n0
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    del g
+    sec = ms / 1e3 / steps
+    ops = float(n) * k * (3 * d + 1)
+    clk = sampler.report()
+    mhz = clk.get("sm_mhz") or 1965.0
+    peak = 148 * 128 * mhz * 1e6 / 1e9             # Gop/s of binary32 add/sub/mul lanes
+    return {"metric": "nearest-centroid assignment, sub-vectors per second", "value": round(world * n / sec / 1e6, 2),
+            "unit": "M sub-vectors/s", "n_gpus": world, "steps": steps, "warmup": args.warmup,
+            "ms_per_step": round(ms / steps, 6), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "encode_4096x4096_d8_k4096",
+                       "describe": "assign the %d sub-vectors (d=8) of a 4096x4096 fp16 weight to a K=4096 fp16 codebook" % n,
+                       "l2": "inputs 33.6 MB in HBM; the codebook tile is re-read from L2 by every block",
+                       "parallelism": "replicas x%d" % world},
+            "gpu_launches": int(launches),
+            "roofline": {"bound": "alu", "achieved": round(ops / sec / 1e9, 1), "peak": round(peak, 1), "unit": "Gop/s",
+                         "frac": round(ops / sec / 1e9 / peak, 4), "peak_source": "derived: 148 SMs x 128 FP32 lanes x SM clock",
+                         "traffic": None},
+            "clocks": clk}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -422,7 +500,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="vqlin", choices=["vqlin", "reference"])
     ap.add_argument("--config", default="qproj",
-                    choices=["qproj", "tiny", "downproj", "smollm", "prefill", "vlen4", "vlen6", "vlen8", "vlen12"])
+                    choices=["qproj", "tiny", "downproj", "smollm", "prefill", "vlen4", "vlen6", "vlen8", "vlen12",
+                             "encode"])
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -442,7 +521,7 @@ def main():
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
         td.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         dist = td
-    line = run_vqlin(args, rank, world, dist)
+    line = run_encode(args, rank, world, dist) if args.config == "encode" else run_vqlin(args, rank, world, dist)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist:

@@ -255,6 +255,22 @@ vqlin_status vqlin_unpack_indices(const vqlin_handle* h, int32_t which, uint32_t
 vqlin_status vqlin_device_error(int32_t* code);
 
 /*
+ * Nearest-centroid assignment, the encoding step that produces the indices the layer
+ * stores (VPTQ page, "Step 3": Q_V(v) = argmin_i ||v - C_i||^2, plain Euclidean distance;
+ * "Residual Vector Quantization": i1 = Q_1(v), i2 = argmin_j ||(v - C1[i1]) - C2_j||^2).
+ *   V    device fp16 [n][d] sub-vectors (d in {4, 6, 8, 12}), finite values
+ *   C1   device fp16 [k1][d] codebook, k1 >= 1
+ *   C2   device fp16 [k2][d] residual codebook, or NULL with k2 = 0
+ *   idx1 device uint32 [n]; idx2 device uint32 [n] when k2 > 0 (else ignored)
+ * Distances are taken in binary32: each difference, square and running sum is rounded
+ * separately (no fused multiply-add), elements in order, centroids from index 0 up; ties keep
+ * the lowest index; the residual is the binary32 difference v - C1[i1].  n = 0 does nothing.
+ * Runs on `stream`; the caller owns every buffer.  No counterpart of this signature on the pages.
+ */
+vqlin_status vqlin_assign(const uint16_t* V, int64_t n, int32_t d, const uint16_t* C1, int32_t k1,
+                          const uint16_t* C2, int32_t k2, uint32_t* idx1, uint32_t* idx2, void* stream);
+
+/*
  * Failure-detection self-test.  Launches on `stream` one thread that waits on a
  * shared-memory mbarrier nothing completes, bounded by `limit_us` microseconds
  * (1..1,000,000) of %globaltimer, exactly like the decode kernel's entry-stream

@@ -86,11 +86,13 @@ vqlin_abi_version = _sig("vqlin_abi_version", C.c_int32, [])
 vqlin_device_error = _sig("vqlin_device_error", _S, [C.POINTER(C.c_int32)])
 vqlin_kernel_launches = _sig("vqlin_kernel_launches", C.c_uint64, [])
 vqlin_selftest_wait_timeout = _sig("vqlin_selftest_wait_timeout", _S, [C.c_int32, C.c_void_p])
+vqlin_assign = _sig("vqlin_assign", _S, [C.c_void_p, C.c_int64, C.c_int32, C.c_void_p, C.c_int32, C.c_void_p,
+                                              C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p])
 
 EXPORTS = ["vqlin_create", "vqlin_destroy", "vqlin_get_info", "vqlin_dequant", "vqlin_gemv", "vqlin_gemm",
            "vqlin_gemm_workspace_size", "vqlin_unpack_indices", "vqlin_status_string", "vqlin_last_error",
            "vqlin_abi_version", "vqlin_device_error", "vqlin_gemv_ws", "vqlin_gemv_workspace_size", "vqlin_gemv_noalloc",
-           "vqlin_kernel_launches", "vqlin_selftest_wait_timeout"]
+           "vqlin_kernel_launches", "vqlin_selftest_wait_timeout", "vqlin_assign"]
 
 
 def device_error() -> int:
