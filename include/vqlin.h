@@ -194,13 +194,18 @@ vqlin_status vqlin_gemv(const vqlin_handle* h, const void* x, vqlin_dtype xt, in
                         void* y, vqlin_dtype yt, void* stream);
 
 /*
- * The same product with a caller-owned scratch buffer: when the layer is too
- * wide for one pass of the tensor-core decode kernel, column chunks are summed
- * in fp32 in `workspace` (>= vqlin_gemv_workspace_size(h, batch) bytes, 256-byte
- * aligned, device memory, not used by another call at the same time) and
- * converted to yt at the end; vqlin_gemv instead has each thread block loop over
- * the chunks itself.  Results agree within the GEMV tolerance (summation order
- * differs).  Errors additionally: WORKSPACE.
+ * The same product with a caller-owned scratch buffer (>= vqlin_gemv_workspace_size(h,
+ * batch) bytes, 256-byte aligned, device memory, not used by another call at the same
+ * time; its contents need not be initialised and are unspecified afterwards).  The
+ * scratch enables the faster kernels:
+ *   - layers with a large single-stage codebook (k1 > 10240, d = 8) and batch <= 4 run
+ *     the codebook-stationary decode, whose blocks each own a slice of the codebook
+ *     and write per-block partial sums here (deterministic: fixed-point row sums);
+ *   - layers too wide for one pass of the tensor-core decode sum column chunks here
+ *     in fp32 and convert to yt at the end (vqlin_gemv instead has each block loop
+ *     over the chunks itself).
+ * Results agree with vqlin_gemv within the GEMV tolerance (summation order differs).
+ * Errors additionally: WORKSPACE.
  */
 vqlin_status vqlin_gemv_ws(const vqlin_handle* h, const void* x, vqlin_dtype xt, int32_t batch,
                            void* y, vqlin_dtype yt, void* workspace, size_t ws_bytes, void* stream);
