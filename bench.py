@@ -418,8 +418,9 @@ def run_reference(args, rank, world):
 def run_encode(args, rank, world, dist):
     """Nearest-centroid assignment of every sub-vector of a 4096x4096 fp16 weight (d = 8, about
     2.1 M sub-vectors) against a K = 4096 codebook (VPTQ's Q_V).  Same timing protocol as the
-    decode bench; the roofline is the CUDA-core ALU: 3d + 1 binary32 operations per
-    (sub-vector, centroid) against 148 SMs x 128 FP32 lanes x the sampled SM clock."""
+    decode bench; the roofline is the CUDA-core ALU: 2d + 1 binary32 lane operations (d
+    subtractions, d fused multiply-adds, one comparison) per (sub-vector, centroid) against
+    148 SMs x 128 FP32 lanes x the sampled SM clock."""
     import torch
     from sparse_compensated_vq_b200 import vqlin
 
@@ -474,7 +475,7 @@ def run_encode(args, rank, world, dist):
         ms = float(t.item())
     del g
     sec = ms / 1e3 / steps
-    ops = float(n) * k * (3 * d + 1)
+    ops = float(n) * k * (2 * d + 1)
     clk = sampler.report()
     mhz = clk.get("sm_mhz") or 1965.0
     peak = 148 * 128 * mhz * 1e6 / 1e9             # Gop/s of binary32 add/sub/mul lanes

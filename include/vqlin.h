@@ -267,8 +267,8 @@ vqlin_status vqlin_device_error(int32_t* code);
  *   C1   device fp16 [k1][d] codebook, k1 >= 1
  *   C2   device fp16 [k2][d] residual codebook, or NULL with k2 = 0
  *   idx1 device uint32 [n]; idx2 device uint32 [n] when k2 > 0 (else ignored)
- * Distances are taken in binary32: each difference, square and running sum is rounded
- * separately (no fused multiply-add), elements in order, centroids from index 0 up; ties keep
+ * Distances are taken in binary32: each difference is one rounded subtraction and the running
+ * sum one fused multiply-add per element, elements in order, centroids from index 0 up; ties keep
  * the lowest index; the residual is the binary32 difference v - C1[i1].  n = 0 does nothing.
  * Runs on `stream`; the caller owns every buffer.  No counterpart of this signature on the pages.
  */

@@ -341,9 +341,10 @@ double oracle_vptq_compression_ratio(int64_t n_elems, int32_t V, int64_t k) {
    VPTQ page, "Step 3: Vector quantization of column n": Q_V(v) = argmin_i ||v - C_i||^2 (plain
    Euclidean distance), and "Residual Vector Quantization": i1 = Q_1(v), v_res = v - C[i1],
    i2 = argmin_j ||v_res - Cres_j||^2.  The pages fix no precision; this restates the decision
-   in the library kernel's precision so both sides take it identically: every difference,
-   square and running sum is one IEEE binary32 operation rounded to nearest (no fused
-   multiply-add; built with -ffp-contract=off), elements in order 0..d-1, centroids scanned
+   in the library kernel's precision so both sides take it identically: every difference is
+   one IEEE binary32 subtraction rounded to nearest and every step of the running sum one
+   binary32 fused multiply-add acc = fma(diff, diff, acc) (C99 fmaf; no other contraction,
+   built with -ffp-contract=off), elements in order 0..d-1, centroids scanned
    from index 0 up, and a centroid replaces the best one only when strictly closer (ties
    keep the lowest index).  v_res is the binary32 difference v - C[i1].  fp16 inputs convert
    to binary32 exactly. */
@@ -356,8 +357,7 @@ static uint32_t nearest_f32(const float* v, int32_t d, const uint16_t* C, int32_
     float acc = 0.0f;
     for (int32_t t = 0; t < d; ++t) {
       volatile float diff = v[t] - f16_to_f32(C[(int64_t)i * d + t]);
-      volatile float sq = diff * diff;
-      acc = acc + sq;
+      acc = fmaf(diff, diff, acc);
     }
     if (i == 0 || acc < best_d) { best = (uint32_t)i; best_d = acc; }
   }

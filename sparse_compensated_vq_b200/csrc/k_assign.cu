@@ -4,11 +4,12 @@
 //
 // One thread per sub-vector holds v in registers; the block stages the codebook tile by tile
 // in shared memory as fp32, so every centroid read is a broadcast.  The decision is taken in
-// binary32 with every difference, square and running sum rounded separately (no fused
-// multiply-add), elements in order 0..d-1, centroids from index 0 up, and a centroid replaces
-// the best one only when strictly closer, so ties keep the lowest index.  The residual is the
-// binary32 difference v - C1[i1].  The work is d subtractions, d multiplications, d additions
-// and one comparison per (sub-vector, centroid): CUDA-core ALU bound.
+// binary32: each difference is one rounded subtraction and the running sum one fused
+// multiply-add per element (acc = fma(diff, diff, acc)), elements in order 0..d-1, centroids
+// from index 0 up, and a centroid replaces the best one only when strictly closer, so ties
+// keep the lowest index.  The residual is the binary32 difference v - C1[i1].  The work is
+// d subtractions, d fused multiply-adds and one comparison per (sub-vector, centroid):
+// CUDA-core ALU bound.
 #include "vqlin_internal.cuh"
 
 namespace vqlin {
@@ -36,7 +37,7 @@ __device__ __forceinline__ void scan_codebook(const __half* __restrict__ C, int 
 #pragma unroll
         for (int t = 0; t < D; ++t) {
           const float diff = __fsub_rn(v[t], c[t]);
-          acc = __fadd_rn(acc, __fmul_rn(diff, diff));
+          acc = __fmaf_rn(diff, diff, acc);
         }
         if ((base == 0 && i == 0) || acc < best_d) { best_d = acc; best_i = (uint32_t)(base + i); }
       }
