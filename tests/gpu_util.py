@@ -66,4 +66,6 @@ def workload(name: str):
         return synth.smollm(8)
     if name == "prefill":
         return synth.prefill(2048)
+    if name.startswith("vlen"):
+        return synth.vlen(int(name[4:]), 16)
     raise KeyError(name)

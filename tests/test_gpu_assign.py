@@ -79,3 +79,16 @@ def test_assign_argument_errors(vq):
     assert vq.vqlin_assign(p, 4, 8, p, 0, None, 0, p, None, None) == 1          # k1 < 1
     assert vq.vqlin_assign(p, 4, 8, p, 4, None, 3, p, p, None) == 1             # k2 > 0 without C2
     assert vq.vqlin_assign(None, 0, 8, None, 4, None, 0, None, None, None) == 0  # n = 0: nothing to do
+
+
+def test_assign_full_encode_workload_sampled(vq):
+    """The bench's encode workload at full size (all 2,097,152 sub-vectors of a 4096x4096 weight,
+    K = 4096), checked against the oracle on 2048 sampled sub-vectors."""
+    rng = synth.rng_for(6)
+    d, k = 8, 4096
+    C1 = synth.f16_bits(rng.normal(0.0, 0.02, (k, d)))
+    V = synth.f16_bits(rng.normal(0.0, 0.02, (4096 * 4096 // d, d)))
+    g, _ = run_assign(vq, V, C1)
+    pick = np.random.default_rng(5).choice(V.shape[0], 2048, replace=False)
+    o, _ = oracle.assign_f32(V[pick], C1)
+    assert (g[pick] == o).all()

@@ -61,13 +61,13 @@ SMALL = small_layers()
 def full_layer(name):
     if name == "tiny":
         return G.workload("tiny")[0]
-    if name in ("qproj", "downproj", "prefill"):
+    if name in ("qproj", "downproj", "prefill") or name.startswith("vlen"):
         return G.workload(name)[0]
     idx = int(name.split(":")[1])
     return G.workload("smollm")[0][idx]
 
 
-FULL = ["tiny", "qproj", "downproj"] + ["smollm:%d" % i for i in range(7)]
+FULL = ["tiny", "qproj", "downproj"] + ["smollm:%d" % i for i in range(7)] + ["vlen6", "vlen12"]
 
 
 # ------------------------------------------------------------------ unpack
