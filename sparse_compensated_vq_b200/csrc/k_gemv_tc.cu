@@ -427,8 +427,9 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
 // so warps overlap each other's memory latency freely.  B fragments are read
 // from shared memory per pair-step, which keeps registers low enough for two
 // blocks per SM.
-template <int NT, int W, bool CB_SMEM, int COPIES>
-__global__ void __launch_bounds__(THREADS, 2) k_gemv_wt(Args a) {
+template <int NT, int W, bool CB_SMEM, int COPIES, int NW>
+__global__ void __launch_bounds__(NW * 32, 16 / NW) k_gemv_wt(Args a) {
+  constexpr int WT_THREADS = NW * 32;   // NW warps per block: 8 (two blocks per SM) or 16 (one)
   constexpr int PS = 16 / NT;
   constexpr int KSV = 4 * PS;
   constexpr int BP = 4 * NT;
@@ -447,17 +448,17 @@ __global__ void __launch_bounds__(THREADS, 2) k_gemv_wt(Args a) {
 
   if (CB_SMEM) {
     const uint4* c1 = reinterpret_cast<const uint4*>(L.cb1);
-    for (int i = threadIdx.x; i < L.k1 * COPIES; i += THREADS) cb1s[i] = __ldg(c1 + i / COPIES);
+    for (int i = threadIdx.x; i < L.k1 * COPIES; i += WT_THREADS) cb1s[i] = __ldg(c1 + i / COPIES);
     if (L.k2) {
       const uint4* c2 = reinterpret_cast<const uint4*>(L.cb2);
-      for (int i = threadIdx.x; i < L.k2 * COPIES; i += THREADS) cb2s[i] = __ldg(c2 + i / COPIES);
+      for (int i = threadIdx.x; i < L.k2 * COPIES; i += WT_THREADS) cb2s[i] = __ldg(c2 + i / COPIES);
     }
   }
   // x (and the accumulator) belong to the previous grid until it completes
   pdl_wait();
   pdl_release();
   const int n_o = L.n_sub_o * 8;
-  for (int i = threadIdx.x; i < BP * n_o; i += THREADS) {
+  for (int i = threadIdx.x; i < BP * n_o; i += WT_THREADS) {
     int b = i / n_o, p = i - b * n_o;
     float v = 0.f;
     if (b < B && p < L.n_ocols) {
@@ -470,7 +471,7 @@ __global__ void __launch_bounds__(THREADS, 2) k_gemv_wt(Args a) {
   // x' hi/lo for every main column, eight columns per thread, loads first
   {
     const int groups = a.xs_cols / 8;
-    for (int i = threadIdx.x; i < B * groups; i += THREADS) {
+    for (int i = threadIdx.x; i < B * groups; i += WT_THREADS) {
       const int b = i / groups, q = (i - b * groups) * 8;
       float v[8];
       if (!L.colmap && a.xt != VQLIN_F32 && q + 8 <= L.n_main && (L.n_in & 7) == 0) {
@@ -516,7 +517,7 @@ __global__ void __launch_bounds__(THREADS, 2) k_gemv_wt(Args a) {
   const int n_side = has_side ? (L.n_out + 7) / 8 : 0;      // sparse / outlier tasks of 8 rows
   const int n_main = n_rt * a.n_kslabs;
   const int total = n_side + n_main;
-  for (int task = blockIdx.x * WARPS + warp; task < total; task += gridDim.x * WARPS) {
+  for (int task = blockIdx.x * NW + warp; task < total; task += gridDim.x * NW) {
     if (task < n_side) {
       // ---- fused sparse correction and outlier block for rows 8*task .. +8 (4 lanes per row)
       const int64_t row = (int64_t)task * 8 + (lane >> 2);
@@ -659,10 +660,12 @@ __global__ void __launch_bounds__(THREADS, 2) k_gemv_wt(Args a) {
 
 template <int NT, int W, bool CB_SMEM, int COPIES>
 static cudaError_t launch_wt_cfg(const Args& args, size_t smem, int grid, cudaStream_t s) {
-  auto k = k_gemv_wt<NT, W, CB_SMEM, COPIES>;
+  // one block per SM (shared memory) runs 16 warps; otherwise two blocks of 8
+  const bool wide = 2 * (smem + 1024) > 227 * 1024;
+  auto k = wide ? k_gemv_wt<NT, W, CB_SMEM, COPIES, 16> : k_gemv_wt<NT, W, CB_SMEM, COPIES, 8>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(k, dim3(grid), THREADS, smem, s, args);
+  return launch_pdl(k, dim3(grid), wide ? 512 : 256, smem, s, args);
 }
 
 template <int NT, int W>
