@@ -5,11 +5,9 @@ compiled library.  Device memory and streams come from PyTorch.  Importing this
 module loads libvqlin.so and raises ImportError if it has not been built
 (``python -m sparse_compensated_vq_b200.build``); there is no fallback.
 
-The functions ``vqlin_create``, ``vqlin_destroy``, ``vqlin_get_info``,
-``vqlin_dequant``, ``vqlin_gemv``, ``vqlin_gemm``,
-``vqlin_gemm_workspace_size``, ``vqlin_unpack_indices``,
-``vqlin_status_string`` and ``vqlin_last_error`` are the C entry points
-themselves.  :class:`VQLinear` wraps them for torch tensors.
+Every function that include/vqlin.h declares is exposed here under its own name
+(the list is ``EXPORTS``) with ctypes argument types; these are the C entry points
+themselves.  :class:`VQLinear` wraps the layer calls for torch tensors.
 """
 from __future__ import annotations
 
