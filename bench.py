@@ -106,6 +106,18 @@ def make_workload(name: str, batch: int) -> Workload:
 
 
 # --------------------------------------------------------------------------- helpers
+def max_over_ranks(value: float, dist) -> float:
+    """The largest `value` over all ranks (a device time: the job is as slow as its slowest rank).
+    Every rank must call it at the same point.  NCCL reduces a CUDA tensor, gloo a CPU one."""
+    if dist is None:
+        return value
+    import torch
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -267,9 +279,7 @@ def run_vqlin(args, rank, world, dist):
     ms = e0.elapsed_time(e1)
     ms_max = ms
     if dist:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
+        ms_max = max_over_ranks(ms, dist)
     del g
 
     # ---- end to end: host buffers, copies inside the timed region, result read each step
@@ -307,9 +317,7 @@ def run_vqlin(args, rank, world, dist):
     del e2e_graphs
     e2e_ms = f0.elapsed_time(f1)
     if dist:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e2e_ms, dist)
     h2d = sum(x.numel() * 2 for x in x_host)
     d2h = sum(y.numel() * 2 for y in y_host)
 
@@ -470,9 +478,7 @@ def run_encode(args, rank, world, dist):
         dist.barrier()
     ms = e0.elapsed_time(e1)
     if dist:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, dist)
     del g
     sec = ms / 1e3 / steps
     ops = float(n) * k * (2 * d + 1)
