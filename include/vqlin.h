@@ -36,10 +36,11 @@
  *   (no residual codebook: the C2 term is absent, not +0; no scale: factor 1).
  *
  * The layer then computes y[b,:] = W x[b,:] (decode, batch 1..16) or
- * Y = X W^T (prefill), with the dequantisation fused into the product
- * (VPTQ page, "The dequantization interface": dequantisation fused into the
- * GEMV for decoding and the GEMM for prefill, so the fp16 weight is never
- * written and re-read).
+ * Y = X W^T (prefill).  The decode fuses the dequantisation into the product,
+ * so the fp16 weight is never written (VPTQ page, "The dequantization
+ * interface": dequantisation fused into the GEMV for decoding).  The prefill
+ * dequantises exactly into the caller's workspace and runs a tcgen05 tensor-core
+ * GEMM on it; the page's fused GEMM for prefill is not built that way here.
  *
  * Packed index format
  * -------------------
