@@ -217,15 +217,18 @@ size_t vqlin_gemv_workspace_size(const vqlin_handle* h, int32_t batch);
  * (a serving loop whose pool already owns the GPU's memory, a path where
  * cudaMalloc's implicit device synchronisation is not allowed, a plug-in that
  * may only touch the buffers it is handed).  It computes what vqlin_gemv_ws
- * computes, but its column-split accumulator is a scratch array built into the
- * library (1 MiB of fp32 per device, held until the process exits) instead of
- * a caller buffer, and it allocates nothing.  Limit: batch * n_out <= 262144,
- * else VQLIN_ERR_UNSUPPORTED.  The first call on a device looks up the array's
- * device address (cudaGetSymbolAddress) and caches it: make that first call
- * outside stream capture.  All calls share the array: calls whose kernels
- * overlap on the GPU race on it, so the caller must serialise them.  The array
- * is cleared on the call's stream before each use.  (No counterpart on the
- * pages: this is an interface convenience.)
+ * computes, with a scratch array built into the library (8 MiB per device, held
+ * until the process exits) in place of a caller buffer, and it allocates
+ * nothing.  The array holds the codebook-stationary partial sums of a 4096-row
+ * layer with a 65536-entry codebook up to batch 4 and the column-split fp32
+ * accumulator of any layer with batch * n_out <= 2097152; a plan that needs more
+ * runs the kernels that need no scratch (as vqlin_gemv does).  Limit: batch *
+ * n_out <= 2097152, else VQLIN_ERR_UNSUPPORTED.  The first call on a device
+ * looks up the array's device address (cudaGetSymbolAddress) and caches it: make
+ * that first call outside stream capture.  All calls share the array: calls
+ * whose kernels overlap on the GPU race on it, so the caller must serialise
+ * them.  What must start at zero is cleared on the call's stream before each
+ * use.  (No counterpart on the pages: this is an interface convenience.)
  */
 vqlin_status vqlin_gemv_noalloc(const vqlin_handle* h, const void* x, vqlin_dtype xt, int32_t batch,
                                 void* y, vqlin_dtype yt, void* stream);
@@ -270,7 +273,11 @@ vqlin_status vqlin_device_error(int32_t* code);
  *   idx1 device uint32 [n]; idx2 device uint32 [n] when k2 > 0 (else ignored)
  * Distances are taken in binary32: each difference is one rounded subtraction and the running
  * sum one fused multiply-add per element, elements in order, centroids from index 0 up; ties keep
- * the lowest index; the residual is the binary32 difference v - C1[i1].  n = 0 does nothing.
+ * the lowest index; the residual is the binary32 difference v - C1[i1].  So idx1 is a nearest
+ * centroid up to rounding: its exact squared distance D satisfies D (1 - e) <= Dmin (1 + e) with
+ * e = (d + 3) 2^-24 and Dmin the exact minimum (idx1 is the exact argmin wherever that minimum
+ * is unique beyond the slack; an exact hit, distance 0, returns its lowest index); idx2 is the
+ * same for v - C1[idx1], up to the additional rounding of that residual.  n = 0 does nothing.
  * Runs on `stream`; the caller owns every buffer.  No counterpart of this signature on the pages.
  */
 vqlin_status vqlin_assign(const uint16_t* V, int64_t n, int32_t d, const uint16_t* C1, int32_t k1,

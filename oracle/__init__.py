@@ -14,6 +14,8 @@ from .oracle import (  # noqa: F401
     dequant_f64,
     gemv_f64,
     vptq_compression_ratio,
-    assign_f32,
+    assign_exact,
+    residual_assign_exact,
+    sqdist_exact,
     OracleError,
 )

@@ -338,47 +338,96 @@ double oracle_vptq_compression_ratio(int64_t n_elems, int32_t V, int64_t k) {
 }
 
 /* ---------------------------------------------------------------- nearest-centroid assignment
-   VPTQ page, "Step 3: Vector quantization of column n": Q_V(v) = argmin_i ||v - C_i||^2 (plain
-   Euclidean distance), and "Residual Vector Quantization": i1 = Q_1(v), v_res = v - C[i1],
-   i2 = argmin_j ||v_res - Cres_j||^2.  The pages fix no precision; this restates the decision
-   in the library kernel's precision so both sides take it identically: every difference is
-   one IEEE binary32 subtraction rounded to nearest and every step of the running sum one
-   binary32 fused multiply-add acc = fma(diff, diff, acc) (C99 fmaf; no other contraction,
-   built with -ffp-contract=off), elements in order 0..d-1, centroids scanned
-   from index 0 up, and a centroid replaces the best one only when strictly closer (ties
-   keep the lowest index).  v_res is the binary32 difference v - C[i1].  fp16 inputs convert
-   to binary32 exactly. */
-static float f16_to_f32(uint16_t h) { return (float)oracle_f16_to_f64(h); }
+   VPTQ page, "Step 3: Vector quantization of column n": Q_V(v) = argmin_i ||v - C_i||^2, the
+   plain Euclidean nearest centroid; "Residual Vector Quantization": i1 = Q_1(v), then the
+   residual v - C[i1] is quantised with the residual codebook, i2 = argmin_j ||(v - C[i1]) -
+   Cres_j||^2.  The pages fix no precision, so this computes the definition exactly: every
+   finite fp16 value is an integer multiple of 2^-24, so a difference of two is an exact integer
+   in those units (at most 42 bits with sign, also for a residual) and a squared distance an exact
+   integer in units of 2^-48 (at most 2^88 for d <= 12, inside __int128).  Centroids are scanned
+   from index 0 up and a later one wins only when strictly closer, so ties keep the lowest index
+   (the pages give no tie rule; this is the reading taken). */
 
-static uint32_t nearest_f32(const float* v, int32_t d, const uint16_t* C, int32_t k) {
+/* A finite fp16 value as an exact integer count of 2^-24. */
+static int64_t f16_units(uint16_t h) {
+  int s = 0, e = 0; int64_t m = 0;
+  if (!f16_split(h, &s, &m, &e)) return 0;   /* callers reject inf/NaN first */
+  /* value = m * 2^e with e >= -24 */
+  int64_t v = m << (e + 24);
+  return s ? -v : v;
+}
+
+/* ||v - c||^2 in units of 2^-48, v given in units of 2^-24, c as fp16. */
+static i128 sqdist_units(const int64_t* v, const uint16_t* c, int32_t d) {
+  i128 acc = 0;
+  for (int32_t t = 0; t < d; ++t) {
+    i128 diff = (i128)v[t] - (i128)f16_units(c[t]);
+    acc += diff * diff;
+  }
+  return acc;
+}
+
+static uint32_t nearest_exact(const int64_t* v, int32_t d, const uint16_t* C, int32_t k) {
   uint32_t best = 0;
-  float best_d = 0.0f;
+  i128 best_d = 0;
   for (int32_t i = 0; i < k; ++i) {
-    float acc = 0.0f;
-    for (int32_t t = 0; t < d; ++t) {
-      volatile float diff = v[t] - f16_to_f32(C[(int64_t)i * d + t]);
-      acc = fmaf(diff, diff, acc);
-    }
-    if (i == 0 || acc < best_d) { best = (uint32_t)i; best_d = acc; }
+    i128 D = sqdist_units(v, C + (int64_t)i * d, d);
+    if (i == 0 || D < best_d) { best = (uint32_t)i; best_d = D; }
   }
   return best;
 }
 
-int oracle_assign_f32(const uint16_t* V, int64_t n, int32_t d, const uint16_t* C1, int32_t k1,
-                      const uint16_t* C2, int32_t k2, uint32_t* idx1, uint32_t* idx2) {
-  float v[64];
-  if (d < 1 || d > 64 || k1 < 1 || (k2 > 0 && !C2)) return ORACLE_BAD_VALUE;
-  for (int64_t e = 0; e < n * d; ++e) if (((V[e] >> 10) & 0x1F) == 31) return ORACLE_BAD_VALUE;
-  for (int64_t e = 0; e < (int64_t)k1 * d; ++e) if (((C1[e] >> 10) & 0x1F) == 31) return ORACLE_BAD_VALUE;
-  for (int64_t e = 0; e < (int64_t)k2 * d; ++e) if (((C2[e] >> 10) & 0x1F) == 31) return ORACLE_BAD_VALUE;
+static int all_finite(const uint16_t* a, int64_t n) {
+  for (int64_t e = 0; e < n; ++e) if (((a[e] >> 10) & 0x1F) == 31) return 0;
+  return 1;
+}
+
+/* idx1[s] = Q_1(V[s]); with a residual codebook also idx2[s] = argmin_j ||(V[s] - C1[idx1[s]]) -
+   C2_j||^2.  V [n][d], C1 [k1][d], C2 [k2][d] as fp16 bits; 1 <= d <= 64. */
+int oracle_assign_exact(const uint16_t* V, int64_t n, int32_t d, const uint16_t* C1, int32_t k1,
+                        const uint16_t* C2, int32_t k2, uint32_t* idx1, uint32_t* idx2) {
+  int64_t v[64];
+  if (d < 1 || d > 64 || k1 < 1 || k2 < 0 || (k2 > 0 && !C2)) return ORACLE_BAD_VALUE;
+  if (!all_finite(V, n * d) || !all_finite(C1, (int64_t)k1 * d) || !all_finite(C2, (int64_t)k2 * d))
+    return ORACLE_BAD_VALUE;
   for (int64_t s = 0; s < n; ++s) {
-    for (int32_t t = 0; t < d; ++t) v[t] = f16_to_f32(V[s * d + t]);
-    const uint32_t i1 = nearest_f32(v, d, C1, k1);
+    for (int32_t t = 0; t < d; ++t) v[t] = f16_units(V[s * d + t]);
+    const uint32_t i1 = nearest_exact(v, d, C1, k1);
     idx1[s] = i1;
     if (k2 > 0) {
-      for (int32_t t = 0; t < d; ++t) { volatile float r = v[t] - f16_to_f32(C1[(int64_t)i1 * d + t]); v[t] = r; }
-      idx2[s] = nearest_f32(v, d, C2, k2);
+      for (int32_t t = 0; t < d; ++t) v[t] -= f16_units(C1[(int64_t)i1 * d + t]);
+      idx2[s] = nearest_exact(v, d, C2, k2);
     }
   }
+  return ORACLE_OK;
+}
+
+/* The residual stage alone, for a given first-stage choice idx1 (each < k1): idx2[s] = argmin_j
+   ||(V[s] - C1[idx1[s]]) - C2_j||^2, exactly. */
+int oracle_residual_assign_exact(const uint16_t* V, int64_t n, int32_t d, const uint16_t* C1, int32_t k1,
+                                 const uint32_t* idx1, const uint16_t* C2, int32_t k2, uint32_t* idx2) {
+  int64_t v[64];
+  if (d < 1 || d > 64 || k1 < 1 || k2 < 1 || !C2) return ORACLE_BAD_VALUE;
+  if (!all_finite(V, n * d) || !all_finite(C1, (int64_t)k1 * d) || !all_finite(C2, (int64_t)k2 * d))
+    return ORACLE_BAD_VALUE;
+  for (int64_t s = 0; s < n; ++s) {
+    if (idx1[s] >= (uint32_t)k1) return ORACLE_BAD_INDEX;
+    for (int32_t t = 0; t < d; ++t) v[t] = f16_units(V[s * d + t]) - f16_units(C1[(int64_t)idx1[s] * d + t]);
+    idx2[s] = nearest_exact(v, d, C2, k2);
+  }
+  return ORACLE_OK;
+}
+
+/* Exact ||v - base - c||^2 in units of 2^-48 as a 128-bit integer split into two halves
+   (base may be NULL for zero); v, base and c are fp16 [d]. */
+int oracle_sqdist_exact(const uint16_t* v, const uint16_t* base, const uint16_t* c, int32_t d, uint64_t* hi,
+                        uint64_t* lo) {
+  int64_t w[64];
+  if (d < 1 || d > 64 || !all_finite(v, d) || !all_finite(c, d) || (base && !all_finite(base, d)))
+    return ORACLE_BAD_VALUE;
+  for (int32_t t = 0; t < d; ++t) w[t] = f16_units(v[t]) - (base ? f16_units(base[t]) : 0);
+  u128 D = (u128)sqdist_units(w, c, d);
+  *hi = (uint64_t)(D >> 64);
+  *lo = (uint64_t)D;
   return ORACLE_OK;
 }

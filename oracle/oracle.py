@@ -78,8 +78,12 @@ def _load():
             lib.oracle_gemv_f64_rows.argtypes = [C.POINTER(_Layer), P, C.c_int32, P, C.c_int64, P]
             lib.oracle_vptq_compression_ratio.restype = C.c_double
             lib.oracle_vptq_compression_ratio.argtypes = [C.c_int64, C.c_int32, C.c_int64]
-            lib.oracle_assign_f32.restype = C.c_int
-            lib.oracle_assign_f32.argtypes = [P, C.c_int64, C.c_int32, P, C.c_int32, P, C.c_int32, P, P]
+            lib.oracle_assign_exact.restype = C.c_int
+            lib.oracle_assign_exact.argtypes = [P, C.c_int64, C.c_int32, P, C.c_int32, P, C.c_int32, P, P]
+            lib.oracle_residual_assign_exact.restype = C.c_int
+            lib.oracle_residual_assign_exact.argtypes = [P, C.c_int64, C.c_int32, P, C.c_int32, P, P, C.c_int32, P]
+            lib.oracle_sqdist_exact.restype = C.c_int
+            lib.oracle_sqdist_exact.argtypes = [P, P, P, C.c_int32, C.POINTER(C.c_uint64), C.POINTER(C.c_uint64)]
             _lib = lib
     return _lib
 
@@ -208,10 +212,11 @@ def vptq_compression_ratio(n_elems: int, V: int, k: int) -> float:
     return float(_load().oracle_vptq_compression_ratio(int(n_elems), int(V), int(k)))
 
 
-def assign_f32(V: np.ndarray, C1: np.ndarray, C2: np.ndarray | None = None):
-    """Nearest-centroid indices of fp16 sub-vectors V [n, d] (uint16 bits) in C1 [k1, d] and,
-    with a residual codebook C2 [k2, d], of v - C1[i1] in C2 (oracle.c: oracle_assign_f32).
-    Returns (idx1, idx2) as uint32 arrays; idx2 is None without C2."""
+def assign_exact(V: np.ndarray, C1: np.ndarray, C2: np.ndarray | None = None):
+    """Exact nearest-centroid indices of fp16 sub-vectors V [n, d] (uint16 bits) in C1 [k1, d]
+    and, with a residual codebook C2 [k2, d], of v - C1[i1] in C2 (oracle.c:
+    oracle_assign_exact; ties keep the lowest index).  Returns (idx1, idx2) as uint32 arrays;
+    idx2 is None without C2."""
     lib = _load()
     V = _c(V, np.uint16)
     C1 = _c(C1, np.uint16)
@@ -228,6 +233,33 @@ def assign_f32(V: np.ndarray, C1: np.ndarray, C2: np.ndarray | None = None):
         k2 = C2.shape[0]
         i2 = np.zeros(n, np.uint32)
         c2p = _ptr(C2)
-    _check(lib.oracle_assign_f32(_ptr(V), C.c_int64(n), C.c_int32(d), _ptr(C1), C.c_int32(k1), c2p, C.c_int32(k2),
-                                 _ptr(i1), _ptr(i2) if i2 is not None else None))
+    _check(lib.oracle_assign_exact(_ptr(V), C.c_int64(n), C.c_int32(d), _ptr(C1), C.c_int32(k1), c2p, C.c_int32(k2),
+                                   _ptr(i1), _ptr(i2) if i2 is not None else None))
     return i1, i2
+
+
+def residual_assign_exact(V: np.ndarray, C1: np.ndarray, idx1: np.ndarray, C2: np.ndarray) -> np.ndarray:
+    """Exact residual-stage indices for a given first-stage choice: argmin_j ||(V[s] -
+    C1[idx1[s]]) - C2_j||^2 (oracle.c: oracle_residual_assign_exact)."""
+    lib = _load()
+    V = _c(V, np.uint16)
+    C1 = _c(C1, np.uint16)
+    C2 = _c(C2, np.uint16)
+    idx1 = _c(idx1, np.uint32)
+    n, d = V.shape
+    i2 = np.zeros(n, np.uint32)
+    _check(lib.oracle_residual_assign_exact(_ptr(V), C.c_int64(n), C.c_int32(d), _ptr(C1), C.c_int32(C1.shape[0]),
+                                            _ptr(idx1), _ptr(C2), C.c_int32(C2.shape[0]), _ptr(i2)))
+    return i2
+
+
+def sqdist_exact(v: np.ndarray, c: np.ndarray, base: np.ndarray | None = None) -> int:
+    """Exact ||v - base - c||^2 of fp16 vectors (uint16 bits, base optional) as an integer count
+    of 2^-48 (oracle.c: oracle_sqdist_exact)."""
+    lib = _load()
+    v = _c(v, np.uint16)
+    c = _c(c, np.uint16)
+    b = _c(base, np.uint16)
+    hi, lo = C.c_uint64(0), C.c_uint64(0)
+    _check(lib.oracle_sqdist_exact(_ptr(v), _ptr(b), _ptr(c), C.c_int32(v.size), C.byref(hi), C.byref(lo)))
+    return (int(hi.value) << 64) | int(lo.value)

@@ -500,6 +500,7 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
   }
   L.n_ls = n_ls;
   L.tstride = tstride;
+  L.tcodes_rows = tcodes.empty() ? 0 : (int32_t)round_up(D->n_out, 16);
   if (up.st == VQLIN_OK) up.st = cuda_status(cudaStreamSynchronize((cudaStream_t)stream), "create sync");
   if (up.st != VQLIN_OK) {
     vqlin_status s = up.st;

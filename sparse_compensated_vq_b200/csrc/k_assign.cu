@@ -9,7 +9,9 @@
 // from index 0 up, and a centroid replaces the best one only when strictly closer, so ties
 // keep the lowest index.  The residual is the binary32 difference v - C1[i1].  The work is
 // d subtractions, d fused multiply-adds and one comparison per (sub-vector, centroid):
-// CUDA-core ALU bound.
+// CUDA-core ALU bound.  Each computed distance lies within (d + 3) 2^-24 of the exact one
+// (relative), so the index returned is a nearest centroid up to that rounding: exactly the
+// argmin wherever the exact minimum is unique beyond it.
 #include "vqlin_internal.cuh"
 
 namespace vqlin {

@@ -540,6 +540,16 @@ cudaError_t launch_gemv_cs(const Layer& L, const void* x, vqlin_dtype xt, int ba
   if (need_words < cap) cap = need_words;
   a.words_cap = cap < 32 ? 32 : cap;
   const size_t smem = cv.total(a.words_cap);
+  // Plan checks on the host, before anything is launched: the carve must lie inside the dynamic
+  // shared memory requested, the word buffer must hold whole 32-word groups, every slot's local
+  // index and row must fit the slice and the row half, and the partial planes must fit the
+  // workspace.  A plan that fails any of them is refused instead of launched.
+  if (smem > smem_max || a.words_cap % 32 != 0 || (int64_t)L.cs_P * L.cs_E < L.k1 ||
+      (int64_t)L.cs_H * L.cs_rpp < L.n_out || (1ll << L.cs_local_bits) <= L.cs_E ||
+      (size_t)(L.cs_E + 1) * copies * 16 > cv.xs || (size_t)L.cs_P * batch * L.n_out * 4 > ws_bytes) {
+    set_error("codebook-stationary decode: inconsistent launch plan (refused)");
+    return cudaErrorInvalidConfiguration;
+  }
   cudaError_t e;
   if (copies == 8) {
     if (L.cs_epw == 3) {

@@ -729,12 +729,17 @@ static cudaError_t launch_nt(const Args& args, bool cb_smem, int copies, size_t 
 
 }  // namespace tcg
 
+// fp32 [batch][n_out] accumulator of the column-split decode (256-byte multiple)
+static size_t gemv_acc_bytes(const Layer& L, int batch) {
+  return ((size_t)batch * L.n_out * 4 + 255) & ~size_t(255);
+}
+
 bool tc_supported(const Layer& L) {
   return L.d == 8 && L.tcodes != nullptr && (L.w == 8 || L.w == 12 || L.w == 16 || L.w == 24 || L.w == 32);
 }
 
 size_t gemv_workspace_bytes(const Layer& L, int batch) {
-  const size_t acc = ((size_t)batch * L.n_out * 4 + 255) & ~size_t(255);
+  const size_t acc = gemv_acc_bytes(L, batch);
   const size_t cs = gemv_cs_workspace_bytes(L, batch);
   return acc > cs ? acc : cs;
 }
@@ -756,6 +761,8 @@ cudaError_t launch_gemv_tc(const Layer& L, const void* x, vqlin_dtype xt, int ba
   if (!tc_supported(L) || batch < 1 || batch > 16) return cudaSuccess;
   const int NT = batch <= 4 ? 1 : (batch <= 8 ? 2 : 4);
   const int KSV = 64 / NT;
+  // the split accumulator needs only [batch][n_out] fp32, whatever else the workspace is sized for
+  const size_t acc_bytes = gemv_acc_bytes(L, batch);
   const int BP = 4 * NT;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -789,6 +796,15 @@ cudaError_t launch_gemv_tc(const Layer& L, const void* x, vqlin_dtype xt, int ba
   const size_t smem = cb_bytes + (size_t)batch * a.xs_cols * 4 + red_bytes + xo_bytes + 64;
   if (smem > smem_max) return cudaSuccess;   // does not fit: caller uses the generic kernel
   const int n_rt = (L.n_out + 15) / 16;
+  // Plan checks on the host: the kernels read index fields of rows up to n_rt * 16 (the layout
+  // pads rows to 16), x' columns up to the staged width (every slab when staged once, one chunk
+  // of ks slabs otherwise), and at most WARPS kernel slabs per chunk.  Refuse a plan that breaks
+  // any of them.
+  if ((int64_t)n_rt * 16 > L.tcodes_rows || a.ks < 1 || a.ks > WARPS || a.rtt * a.ks != WARPS ||
+      a.xs_cols < (a.xs_all ? all_cols : chunk_cols) || (int64_t)a.n_chunks * a.ks < a.n_kslabs) {
+    set_error("tensor-core decode: inconsistent launch plan (refused)");
+    return cudaErrorInvalidConfiguration;
+  }
   const int n_rg = (n_rt + a.rtt - 1) / a.rtt;
   // ---- warp-task kernel: needs an fp32 accumulator (y itself, or the caller's workspace)
   //      and x' for every column next to the codebooks.  When one block task already
@@ -797,7 +813,7 @@ cudaError_t launch_gemv_tc(const Layer& L, const void* x, vqlin_dtype xt, int ba
   if (a.n_chunks > 1 || n_rg > sms) {
     float* acc = nullptr;
     if (yt == VQLIN_F32) acc = reinterpret_cast<float*>(y);
-    else if (ws && ws_bytes >= gemv_workspace_bytes(L, batch)) acc = reinterpret_cast<float*>(ws);
+    else if (ws && ws_bytes >= acc_bytes) acc = reinterpret_cast<float*>(ws);
     int wcopies = 0;
     bool wcb = false;
     for (int c = 8; c >= 1; c >>= 1) {
@@ -836,7 +852,7 @@ cudaError_t launch_gemv_tc(const Layer& L, const void* x, vqlin_dtype xt, int ba
   a.split = 0;
   if (a.n_chunks > 1) {
     if (yt == VQLIN_F32) { a.split = 1; a.acc = reinterpret_cast<float*>(y); }
-    else if (ws && ws_bytes >= gemv_workspace_bytes(L, batch)) { a.split = 1; a.acc = reinterpret_cast<float*>(ws); }
+    else if (ws && ws_bytes >= acc_bytes) { a.split = 1; a.acc = reinterpret_cast<float*>(ws); }
     // otherwise every task loops over the chunks itself (no scratch needed)
   }
   const int n_tasks = a.split ? n_rg * a.n_chunks : n_rg;

@@ -6,26 +6,35 @@
 // activations), a latency-critical path where cudaMalloc's implicit device
 // synchronisation is not allowed, or a plug-in inside another framework that
 // may only touch buffers it is handed.  vqlin_gemv_ws needs a caller-supplied
-// scratch buffer for its column-split fp32 accumulation; this entry point
-// instead uses a fixed-size scratch array compiled into the library, so the
-// caller passes only x and y.
+// scratch buffer; this entry point instead uses a fixed-size scratch array
+// compiled into the library, so the caller passes only x and y.
 //
-// The scratch is a file-scope __device__ array of kScratchFloats floats (1 MiB).
-// Every GPU that loads the library holds it until the process exits.  Host code
-// cannot use the array's name as a device address, so the first call on each
-// device looks the address up with cudaGetSymbolAddress (with that device
-// current) and caches it; make that first call outside any stream capture.
-// All calls share the one array: calls whose kernels overlap on the GPU (for
-// example on two streams) race on it and must be serialised by the caller.  The
-// accumulator is cleared on the call's stream before every use, so what a
-// previous call left there does not leak into the result.
+// The scratch is a file-scope __device__ array of kScratchBytes (8 MiB).  Every
+// GPU that loads the library holds it until the process exits.  It is sized so
+// that the kernels vqlin_gemv_ws would pick also run here for the layers this
+// library targets: the codebook-stationary decode of a 4096-row layer with a
+// 65536-entry codebook keeps 74 fp32 partial-sum planes per batch row (4.6 MiB at
+// batch 4), and the column-split decode keeps one fp32 accumulator of
+// batch * n_out floats.  A layer whose plan needs more than the array holds
+// falls back to the kernels that need no scratch, as vqlin_gemv does; a layer
+// with batch * n_out above kScratchBytes / 4 is refused with UNSUPPORTED.
+//
+// Host code cannot use the array's name as a device address, so the first call
+// on each device looks the address up with cudaGetSymbolAddress (with that
+// device current) and caches it; make that first call outside any stream
+// capture.  All calls share the one array: calls whose kernels overlap on the
+// GPU (for example on two streams) race on it and must be serialised by the
+// caller.  Whatever part must start at zero is cleared on the call's stream
+// before every use, so what a previous call left there does not leak into the
+// result.
 #include <mutex>
 
 #include "vqlin_internal.cuh"
 
 namespace vqlin {
 
-constexpr size_t kScratchFloats = 262144;   // batch * n_out must not exceed this (1 MiB of fp32)
+constexpr size_t kScratchBytes = 8u << 20;               // 8 MiB
+constexpr size_t kScratchFloats = kScratchBytes / sizeof(float);
 static __device__ __align__(256) float g_gemv_scratch[kScratchFloats];
 
 namespace {
@@ -79,7 +88,6 @@ extern "C" vqlin_status vqlin_gemv_noalloc(const vqlin_handle* h, const void* x,
   void* scratch = nullptr;
   vqlin_status st = scratch_address(&scratch);
   if (st) return st;
-  return cuda_status(launch_gemv(h->L, x, xt, batch, y, yt, scratch, kScratchFloats * sizeof(float),
-                                 (cudaStream_t)stream),
+  return cuda_status(launch_gemv(h->L, x, xt, batch, y, yt, scratch, kScratchBytes, (cudaStream_t)stream),
                      "gemv (no-alloc) launch");
 }

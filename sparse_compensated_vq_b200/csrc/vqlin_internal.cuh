@@ -39,6 +39,7 @@ struct Layer {
   // fields of sub-vectors 64*slab + 4*ps + t (ps = 0..15), packed LSB-first.
   const uint8_t* tcodes;
   int32_t n_ls;                         // layout slabs per row
+  int32_t tcodes_rows;                  // rows allocated in tcodes (n_out rounded up to 16)
   int64_t tstride;                      // bytes per row = n_ls * 8 * w
   // Codebook-stationary layout (large single-stage codebooks, d = 8; null otherwise):
   // block c = p * cs_H + h owns codebook slice p (entries [p*cs_E, (p+1)*cs_E), cs_E < 1024)

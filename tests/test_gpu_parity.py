@@ -45,6 +45,8 @@ def small_layers():
         dict(n_out=70, n_in=300, d=12, k1=4096, bits1=12, k2=256, bits2=8, nnz=90, n_ocols=10, ko=64, bits_o=6),
         dict(n_out=19, n_in=96, d=6, k1=1, bits1=1, nnz=5),
         dict(n_out=40, n_in=192, d=12, k1=512, bits1=9, col_scale=True, nnz=30),
+        # residual codebook + outlier block with n_in % 8 == 0, so the prefill GEMM covers both
+        dict(n_out=96, n_in=208, d=4, k1=100, bits1=7, k2=30, bits2=5, col_scale=True, nnz=60, n_ocols=6, ko=50, bits_o=6),
     ]
     out = []
     for t, kw in enumerate(specs):
@@ -175,8 +177,7 @@ def test_gemv_dtypes(vq, xdt, ydt):
     G.assert_close(y, oracle.gemv_f64(L, synth.bits_to_f64(xb, xdt)), ydt, "dtypes")
 
 
-@pytest.mark.parametrize("name", FULL)
-@pytest.mark.parametrize("batch", [1, 16])
+@pytest.mark.parametrize("name,batch", [(n, b) for n in FULL for b in (1, 16)] + [("downproj", 4)])
 def test_gemv_full(vq, name, batch):
     L = full_layer(name)
     if name.startswith("smollm"):
@@ -266,7 +267,7 @@ def run_gemm(vq, L, Xbits, xdt, ydt):
     return G.to_f64(Y)
 
 
-@pytest.mark.parametrize("t", [0, 1, 4, 10, 11])
+@pytest.mark.parametrize("t", [0, 1, 2, 4, 10, 11, 12])
 @pytest.mark.parametrize("M", [1, 77, 256])
 def test_gemm_small(vq, t, M):
     L = SMALL[t]
@@ -331,8 +332,8 @@ def test_device_pointers_create(vq):
 
 
 # ------------------------------------------------------------------ gemv with a caller workspace (split columns)
-@pytest.mark.parametrize("name,batch,ydt", [("downproj", 1, "f16"), ("downproj", 16, "bf16"), ("smollm:6", 8, "f16"),
-                                            ("qproj", 4, "f16"), ("smollm:0", 1, "f32")])
+@pytest.mark.parametrize("name,batch,ydt", [("downproj", 1, "f16"), ("downproj", 4, "f16"), ("downproj", 16, "bf16"),
+                                            ("smollm:6", 8, "f16"), ("qproj", 4, "f16"), ("smollm:0", 1, "f32")])
 def test_gemv_ws_full(vq, name, batch, ydt):
     import torch
     L = full_layer(name)
@@ -441,3 +442,18 @@ def test_codebook_stationary_is_deterministic(vq):
     x = G.torch_x(xb[:4], "f16")
     ys = [m.gemv_ws(x, out_dtype=torch.float32).cpu().numpy().view(np.uint32) for _ in range(3)]
     assert (ys[0] == ys[1]).all() and (ys[0] == ys[2]).all()
+
+
+# ------------------------------------------------------------------ bit accounting of a created layer
+def test_library_info_matches_the_vptq_worked_example(vq):
+    """The library's own accounting for a 4096x4096 layer with V = 8 and k = 256 (VPTQ page,
+    "Compression ratio calculation", the example taken from its section 2.2): ratio 15.97 and
+    about 1.002 bits per weight, as printed there."""
+    g = json.load(open(os.path.join(GOLDEN, "vptq_compression_example.json")))
+    rng = np.random.default_rng(4096)
+    L = synth.random_layer(rng, 4096, 4096, g["V"], g["k"], 8, row_scale=False, nnz=0)
+    info = vq.VQLinear(L).info()
+    assert round(info["vptq_compression_ratio"], g["ratio_printed_decimals"]) == g["ratio_printed"]
+    assert round(info["vptq_bits_per_weight"], g["bits_printed_decimals"]) == g["bits_printed"]
+    assert abs(16.0 / info["vptq_compression_ratio"] - info["vptq_bits_per_weight"]) < 1e-12
+    assert info["index_bytes"] == 4096 * 512 and info["codebook_bytes"] == 2 * 8 * 256

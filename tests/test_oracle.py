@@ -336,30 +336,75 @@ def test_malformed_csr_is_reported():
 
 # ---------------------------------------------------------------- nearest-centroid assignment
 # VPTQ page, "Step 3": Q_V(v) = argmin_i ||v - C_i||^2; "Residual Vector Quantization":
-# i2 = argmin_j ||(v - C1[i1]) - Cres_j||^2.  The oracle takes the decision in binary32; these
-# pins hold it to the exact (rational) argmin wherever binary32 cannot change the answer.
-U32 = 2.0 ** -24
+# i2 = argmin_j ||(v - C1[i1]) - Cres_j||^2.  The oracle computes these exactly (integer units of
+# 2^-24), ties to the lowest index.  The pins: an independent exact-rational brute force, the
+# one-dimensional case against numpy's argmin on exact float64 differences, a case that float64
+# squares cannot decide, exact hits and ties, scaling invariance, constructed residual pairs, and
+# the oracle's own exact distances against the brute force.
 
 
-def _exact_sqdist(v_bits, c_bits):
-    return sum(((exact.f16_frac(int(a)) - exact.f16_frac(int(b))) ** 2 for a, b in zip(v_bits, c_bits)), Fraction(0))
+def _exact_sqdist(v_bits, c_bits, base_bits=None):
+    base = [0] * len(v_bits) if base_bits is None else [exact.f16_frac(int(b)) for b in base_bits]
+    return sum(((exact.f16_frac(int(a)) - o - exact.f16_frac(int(b))) ** 2
+                for a, o, b in zip(v_bits, base, c_bits)), Fraction(0))
+
+
+def _brute_argmin(v_bits, C, base_bits=None):
+    dist = [_exact_sqdist(v_bits, C[i], base_bits) for i in range(len(C))]
+    return min(range(len(C)), key=lambda i: (dist[i], i))
 
 
 @pytest.mark.parametrize("d", [4, 6, 8, 12])
-def test_assign_matches_exact_argmin_where_binary32_cannot_decide_otherwise(d):
+def test_assign_is_the_exact_argmin(d):
     rng = np.random.default_rng(300 + d)
-    k, n = 37, 25
-    C = synth.f16_bits(rng.normal(0, 1, (k, d)))
+    k1, k2, n = 37, 11, 25
+    C1 = synth.f16_bits(rng.normal(0, 1, (k1, d)))
+    C2 = synth.f16_bits(rng.normal(0, 0.3, (k2, d)))
     V = synth.f16_bits(rng.normal(0, 1, (n, d)))
-    i1, _ = oracle.assign_f32(V, C)
-    tol = Fraction(2 * (d + 3)) * Fraction(U32)           # relative error of one binary32 distance
+    i1, i2 = oracle.assign_exact(V, C1, C2)
     for s in range(n):
-        dist = [_exact_sqdist(V[s], C[i]) for i in range(k)]
-        best = min(dist)
-        assert dist[int(i1[s])] <= best * (1 + 2 * tol)    # the pick is (near-)optimal
-        order = sorted(range(k), key=lambda i: (dist[i], i))
-        if dist[order[1]] > best * (1 + 2 * tol):          # unique beyond rounding: must match
-            assert int(i1[s]) == order[0]
+        a = _brute_argmin(V[s], C1)
+        assert int(i1[s]) == a
+        assert int(i2[s]) == _brute_argmin(V[s], C2, base_bits=C1[a])
+    # the residual stage for a prescribed first choice
+    forced = rng.integers(0, k1, n).astype(np.uint32)
+    r2 = oracle.residual_assign_exact(V, C1, forced, C2)
+    for s in range(n):
+        assert int(r2[s]) == _brute_argmin(V[s], C2, base_bits=C1[forced[s]])
+
+
+def test_sqdist_is_exact():
+    rng = np.random.default_rng(310)
+    for d in (1, 4, 8, 12):
+        v, c, b = (synth.f16_bits(rng.normal(0, 100, d)) for _ in range(3))
+        assert Fraction(oracle.sqdist_exact(v, c), 2 ** 48) == _exact_sqdist(v, c)
+        assert Fraction(oracle.sqdist_exact(v, c, b), 2 ** 48) == _exact_sqdist(v, c, b)
+    # the extremes of the format: largest finite values of opposite sign, smallest subnormal
+    v = np.array([0x7BFF, 0x0001, 0x8001], np.uint16)
+    c = np.array([0xFBFF, 0x8001, 0x0001], np.uint16)
+    assert Fraction(oracle.sqdist_exact(v, c), 2 ** 48) == _exact_sqdist(v, c)
+
+
+def test_assign_one_dimension_is_the_nearest_value():
+    """d = 1: the nearest scalar; fp16 differences are exact in float64, so numpy's argmin of
+    |v - c| (first index on ties) is the exact answer."""
+    rng = np.random.default_rng(311)
+    C = synth.f16_bits(rng.normal(0, 1, (200, 1)))
+    V = synth.f16_bits(rng.normal(0, 1.2, (500, 1)))
+    i1, _ = oracle.assign_exact(V, C)
+    cv = C[:, 0].view(np.float16).astype(np.float64)
+    vv = V[:, 0].view(np.float16).astype(np.float64)
+    assert (i1 == np.argmin(np.abs(vv[:, None] - cv[None, :]), axis=1)).all()
+
+
+def test_assign_decides_where_double_precision_squares_tie():
+    """||(0,0) - (1024, 2^-24)||^2 = 2^20 + 2^-48 rounds to 2^20 in float64, a tie with (1024, 0);
+    exactly, (1024, 0) is closer."""
+    V = synth.f16_bits(np.array([[0.0, 0.0]]))
+    C = synth.f16_bits(np.array([[1024.0, 2.0 ** -24], [1024.0, 0.0]]))
+    f = C.view(np.float16).astype(np.float64)
+    assert (f ** 2).sum(axis=1)[0] == (f ** 2).sum(axis=1)[1]
+    assert oracle.assign_exact(V, C)[0].tolist() == [1]
 
 
 def test_assign_exact_hits_and_ties_take_the_lowest_index():
@@ -368,12 +413,24 @@ def test_assign_exact_hits_and_ties_take_the_lowest_index():
     base = synth.f16_bits(rng.normal(0, 1, (10, d)))
     C = np.concatenate([base, base[[3, 7]], base]).astype(np.uint16)   # duplicates at 10, 11 and 12..21
     V = base[[3, 7, 0, 9]]
-    i1, _ = oracle.assign_f32(V, C)
+    i1, _ = oracle.assign_exact(V, C)
     assert i1.tolist() == [3, 7, 0, 9]
     # equidistant centroids: v halfway (exactly) between two candidates
     C2 = synth.f16_bits(np.array([[0, 0, 0, 0], [2, 0, 0, 0], [1, 0, 0, 1.5], [1, 0, 0, -1.5]]))
     V2 = synth.f16_bits(np.array([[1, 0, 0, 0]]))
-    assert oracle.assign_f32(V2, C2)[0].tolist() == [0]
+    assert oracle.assign_exact(V2, C2)[0].tolist() == [0]
+    C3 = C2[[1, 0, 2, 3]]                      # the same tie with the candidates swapped
+    assert oracle.assign_exact(V2, C3)[0].tolist() == [0]
+
+
+def test_assign_invariant_under_power_of_two_scaling():
+    rng = np.random.default_rng(312)
+    d = 8
+    Cf = rng.normal(0, 1, (64, d)).astype(np.float16).astype(np.float64)
+    Vf = rng.normal(0, 1, (300, d)).astype(np.float16).astype(np.float64)
+    a, _ = oracle.assign_exact(synth.f16_bits(Vf), synth.f16_bits(Cf))
+    b, _ = oracle.assign_exact(synth.f16_bits(Vf * 4.0), synth.f16_bits(Cf * 4.0))
+    assert (a == b).all()
 
 
 def test_residual_stage_recovers_constructed_pairs():
@@ -390,7 +447,7 @@ def test_residual_stage_recovers_constructed_pairs():
     pairs = [(a, b) for a in range(k1) for b in range(k2)]
     f = lambda h: h.view(np.float16).astype(np.float64)
     V = synth.f16_bits(np.array([f(C1[a]) + f(C2[b]) for a, b in pairs]))
-    i1, i2 = oracle.assign_f32(V, C1, C2)
+    i1, i2 = oracle.assign_exact(V, C1, C2)
     assert list(zip(i1.tolist(), i2.tolist())) == pairs
 
 
@@ -398,4 +455,4 @@ def test_assign_rejects_non_finite_input():
     C = synth.f16_bits(np.ones((2, 4)))
     V = np.array([[0x7C00, 0, 0, 0]], dtype=np.uint16)     # +inf
     with pytest.raises(oracle.OracleError):
-        oracle.assign_f32(V, C)
+        oracle.assign_exact(V, C)

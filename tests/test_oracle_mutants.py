@@ -27,11 +27,14 @@ MUTANTS = {
     "outlier_codebook": ("*e1 = L->cbo + (int64_t)io * d + (p % d);",
                          "*e1 = L->cb1 + (int64_t)(io % L->k1) * d + (p % d);"),
     "col_scale_dropped": ("if (L->cs) v = v * oracle_f16_to_f64(L->cs[j]);", ";"),
-    "assign_ties_highest": ("if (i == 0 || acc < best_d) {", "if (i == 0 || acc <= best_d) {"),
-    "assign_residual_dropped": ("volatile float r = v[t] - f16_to_f32(C1[(int64_t)i1 * d + t]); v[t] = r;",
-                                "volatile float r = v[t]; v[t] = r;"),
-    "assign_element_skewed": ("volatile float diff = v[t] - f16_to_f32(C[(int64_t)i * d + t]);",
-                              "volatile float diff = v[t] - f16_to_f32(C[(int64_t)i * d + (t + 1) % d]);"),
+    "assign_ties_highest": ("if (i == 0 || D < best_d) {", "if (i == 0 || D <= best_d) {"),
+    "assign_residual_dropped": ("      for (int32_t t = 0; t < d; ++t) v[t] -= f16_units(C1[(int64_t)i1 * d + t]);\n",
+                                "\n"),
+    "assign_element_skewed": ("i128 diff = (i128)v[t] - (i128)f16_units(c[t]);",
+                              "i128 diff = (i128)v[t] - (i128)f16_units(c[(t + 1) % d]);"),
+    "assign_sum_not_difference": ("i128 diff = (i128)v[t] - (i128)f16_units(c[t]);",
+                                  "i128 diff = (i128)v[t] + (i128)f16_units(c[t]);"),
+    "assign_units_truncated": ("  int64_t v = m << (e + 24);", "  int64_t v = (m << (e + 24)) >> 4 << 4;"),
 }
 
 

@@ -47,14 +47,38 @@ def test_noalloc_matches_workspace_variant_twice_in_a_row():
         G.assert_close(G.to_f64(y), G.to_f64(y_ref), "f16", "no-alloc call %d" % call)
 
 
+@pytest.mark.parametrize("batch", [1, 4])
+def test_noalloc_headline_layer_against_the_oracle(batch):
+    """The 4096x4096 layer with a 65536-entry codebook: the built-in scratch holds its
+    codebook-stationary partial sums, so the call runs the same two kernels as
+    vqlin_gemv_ws (not the scratch-free fallback) and matches the CPU oracle."""
+    import torch
+    import oracle
+    from sparse_compensated_vq_b200 import vqlin
+    L, xb = synth.qproj(4)
+    m = vqlin.VQLinear(L)
+    stream = torch.cuda.current_stream().cuda_stream
+    x = G.torch_x(xb[:batch], "f16")
+    y = torch.full((batch, L.n_out), float("nan"), dtype=torch.float32, device="cuda")
+    for call in range(2):
+        n0 = vqlin.vqlin_kernel_launches()
+        vqlin.check(vqlin.vqlin_gemv_noalloc(m.handle, x.data_ptr(), vqlin.VQLIN_F16, batch, y.data_ptr(),
+                                             vqlin.VQLIN_F32, stream), "gemv_noalloc")
+        assert vqlin.vqlin_kernel_launches() - n0 == 2      # codebook-stationary grid + finalize
+        torch.cuda.synchronize()
+        assert vqlin.device_error() == 0
+        ref = oracle.gemv_f64(L, synth.bits_to_f64(xb[:batch], "f16"))
+        G.assert_close(G.to_f64(y), ref, "f32", "no-alloc qproj B=%d call %d" % (batch, call))
+
+
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     import torch
     from sparse_compensated_vq_b200 import vqlin
     rng = np.random.default_rng(7)
-    L = synth.random_layer(rng, 17000, 64, 8, 16, 4, row_scale=False, nnz=0)   # 16 * 17000 > 262144
+    L = synth.random_layer(rng, 131073, 64, 8, 16, 4, row_scale=False, nnz=0)   # 16 * 131073 > 2097152
     m = vqlin.VQLinear(L)
     x = torch.zeros((16, 64), dtype=torch.float16, device="cuda")
-    y = torch.zeros((16, 17000), dtype=torch.float16, device="cuda")
+    y = torch.zeros((16, 131073), dtype=torch.float16, device="cuda")
     st = vqlin.vqlin_gemv_noalloc(m.handle, x.data_ptr(), vqlin.VQLIN_F16, 16, y.data_ptr(), vqlin.VQLIN_F16, None)
     assert st == vqlin.VQLIN_ERR_UNSUPPORTED
     assert b"scratch" in vqlin.vqlin_last_error()
