@@ -96,6 +96,21 @@ def make_workload(name: str, batch: int) -> Workload:
         L, Xb = synth.prefill(2048)
         return Workload("prefill_2048x4096x4096_d8_k65536", [L], [Xb], [(0, 2048)], "gemm",
                         "X 2048x4096 bf16 times the q_proj-shaped VQ weight, bf16 Y")
+    if name == "qproj_sym":
+        L, xb = synth.qproj_sym(batch)
+        return Workload("llama2_7b_qproj_4096x4096_d8_k65536_symmetric_b%d" % batch, [L], [xb], [(0, batch)], "gemv",
+                        "4096x4096, d=8, symmetric codebook: 16384 stored fp16 entries addressed as 65536 "
+                        "(16-bit codes), fp16 row+col scales, 1%% CSR outliers, fp16 x/y, batch %d" % batch)
+    if name == "qproj_groups":
+        L, xb = synth.qproj_groups(batch)
+        return Workload("llama2_7b_qproj_4096x4096_d8_k65536_groups4_b%d" % batch, [L], [xb], [(0, batch)], "gemv",
+                        "4096x4096, d=8, 4 codebook groups of 65536 fp16 entries (16-bit codes), fp16 row+col "
+                        "scales, 1%% CSR outliers, fp16 x/y, batch %d" % batch)
+    if name == "smollm_vsr":
+        Ls, xs = synth.smollm_vsr(batch)
+        return Workload("smollm2_1.7b_layer_7linears_d8_k256_vsr_b%d" % batch, Ls, xs, [(i, batch) for i in range(7)],
+                        "gemv", "7 linears of a SmolLM2-1.7B layer, d=8, K=256, 2%% of the sub-vectors as VSR blocks "
+                        "(position probability ~ |z|^4), bf16 x, batch %d" % batch)
     if name.startswith("vlen"):
         d = int(name[4:])
         L, xb = synth.vlen(d, batch)
@@ -349,7 +364,7 @@ def run_vqlin(args, rank, world, dist):
         achieved = flops_step / per_launch_s / 1e12
         line["roofline"] = {"bound": "tensor", "achieved": round(achieved, 2), "peak": bf16_peak, "unit": "TFLOP/s",
                             "frac": round(achieved / bf16_peak, 4), "peak_source": peak_src + " bf16 (fp16 same rate)",
-                            "traffic": recorded_traffic(wl.name), "kernel": "vqlin gemm step (dequant + convert + GEMM)"}
+                            "traffic": recorded_traffic(wl.name), "kernel": "vqlin gemm step (bf16->fp16 activation convert + GEMM with weight tiles dequantised in shared memory)"}
     line["e2e"] = {"value": round(world * bytes_step * n_e2e / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
                    "us_per_step": round(e2e_ms * 1e3 / n_e2e, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     line["clocks"] = sampler.report()
@@ -508,6 +523,7 @@ def main():
     ap.add_argument("--impl", default="vqlin", choices=["vqlin", "reference"])
     ap.add_argument("--config", default="qproj",
                     choices=["qproj", "tiny", "downproj", "smollm", "prefill", "vlen4", "vlen6", "vlen8", "vlen12",
+                             "qproj_sym", "qproj_groups", "smollm_vsr",
                              "encode"])
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

@@ -36,11 +36,13 @@
  *   (no residual codebook: the C2 term is absent, not +0; no scale: factor 1).
  *
  * The layer then computes y[b,:] = W x[b,:] (decode, batch 1..16) or
- * Y = X W^T (prefill).  The decode fuses the dequantisation into the product,
- * so the fp16 weight is never written (VPTQ page, "The dequantization
- * interface": dequantisation fused into the GEMV for decoding).  The prefill
- * dequantises exactly into the caller's workspace and runs a tcgen05 tensor-core
- * GEMM on it; the page's fused GEMM for prefill is not built that way here.
+ * Y = X W^T (prefill).  Both fuse the dequantisation into the product, so the
+ * fp16 weight is never written to global memory (VPTQ page, "The dequantization
+ * interface": dequantisation fused into the GEMV for decoding and the GEMM for
+ * prefill): the prefill dequantises each weight tile in shared memory and feeds
+ * it to the tcgen05 tensor cores.  (Layers with a residual codebook, an outlier
+ * block or d != 8 take a two-phase prefill instead: exact dequantisation into the
+ * caller's workspace, then the tensor-core GEMM.)
  *
  * Packed index format
  * -------------------
@@ -135,6 +137,36 @@ typedef struct {
   const int32_t* row_ptr;     /* [n_out + 1], row_ptr[0] = 0, non-decreasing, = nnz at end */
   const int32_t* col_idx;     /* [nnz], strictly increasing within a row, in [0, n_in) */
   const uint16_t* values;     /* fp16 [nnz], finite                                    */
+
+  /* VSR: a structured sparse correction by whole sub-vectors (SCVQ summary: the important
+     weights sit contiguously within rows, in line with VQ's sub-vector grouping, and are kept
+     in a structured sparse format, "VSR").  The pages give no layout; this library's reading is
+     a row-compressed format whose unit is one main-column sub-vector: block b of row i covers
+     sub-vector s = vsr_pos[b], i.e. the main columns q = s*d .. s*d + d - 1, and REPLACES every
+     one of its elements: W[i, main column q] = vsr_values[b*d + q - s*d] (a tail sub-vector's
+     values past the last main column are ignored).  A block may not share an element with the
+     CSR matrix (INVALID_DATA).  Per block: one 4-byte position and d fp16 values, instead of d
+     (value, column) pairs. */
+  int64_t vsr_nblocks;        /* 0 <= vsr_nblocks; 0 allows NULL arrays                 */
+  const int32_t* vsr_row_ptr; /* [n_out + 1] over blocks, [0] = 0, non-decreasing, = vsr_nblocks at end */
+  const int32_t* vsr_pos;     /* [vsr_nblocks], strictly increasing within a row, in [0, n_sub) */
+  const uint16_t* vsr_values; /* fp16 [vsr_nblocks][d], finite                           */
+
+  /* Codebook groups (VPTQ page, "Outlier Elimination", on group partitioning: the non-outlier
+     weights split into group_num groups with independent codebooks).  The pages do not say how
+     groups are formed; this library's reading: the main sub-vector positions of every row form
+     n_groups contiguous ranges of g = ceil(n_sub / n_groups) positions, position s decodes with
+     codebook s / g, and codebook1 (and codebook2) hold the n_groups codebooks back to back,
+     [n_groups][k][d].  0 or 1: one codebook.  1 <= n_groups <= n_sub. */
+  int32_t n_groups;
+
+  /* Symmetric codebook (SCVQ summary: symmetry constraints shrink the codebook, to a quarter of
+     its size).  The pages do not name the symmetry; this library's reading: each codebook1 stores
+     k1 / 4 base entries, and entry t * (k1 / 4) + b of the k1 addressed by the indices is base
+     entry b under sign pattern t: t = 0 all +, t = 1 all -, t = 2 odd elements negated, t = 3 even
+     elements negated (a group of four sign patterns; negation is exact in fp16).  0: none;
+     1: this symmetry (needs k1 % 4 == 0; the residual and outlier codebooks stay plain). */
+  int32_t cb_symmetry;
 } vqlin_desc;
 
 /* Sizes and bit accounting of a created layer. */
@@ -142,16 +174,19 @@ typedef struct {
   int32_t n_out, n_in, d, n_sub, n_sub_o, n_ocols;
   int64_t nnz;
   int64_t index_bytes;        /* packed main + outlier fields, rows packed without padding */
-  int64_t codebook_bytes;     /* 2 * d * (k1 + k2 + ko)                                 */
+  int64_t codebook_bytes;     /* stored codebooks: 2 * d * (n_groups * (k1s + k2) + ko), k1s =
+                                 k1 / 4 with a symmetric codebook, else k1                */
   int64_t scale_bytes;        /* 2 * (n_out if row scales) + 2 * (n_in if column scales) */
   int64_t sparse_bytes;       /* CSR: nnz * (2 value + 4 column) + 4 * (n_out + 1)      */
   /* VPTQ page, "Compression ratio calculation": original fp16 bits divided by
      (codebook bits + index bits); equivalent bit width = 16 / ratio.  These two
-     use exactly that formula (main codebook and main indices only). */
+     use exactly that formula over the main codebooks as stored (n_groups * k1s
+     entries) and the main indices only. */
   double vptq_compression_ratio;
   double vptq_bits_per_weight;
-  /* everything the layer stores (indices, all codebooks, scales, CSR), in bits per weight */
+  /* everything the layer stores (indices, all codebooks, scales, CSR, VSR), in bits per weight */
   double total_bits_per_weight;
+  int64_t vsr_bytes;          /* VSR: 4 * (n_out + 1) + vsr_nblocks * (4 + 2 d), 0 without VSR */
 } vqlin_info;
 
 /*
@@ -237,7 +272,12 @@ vqlin_status vqlin_gemv_noalloc(const vqlin_handle* h, const void* x, vqlin_dtyp
  * Prefill: Y[m*n_out + i] = sum_j W[i,j] * X[m*n_in + j] for 0 <= m < M.
  * X: device [M][n_in] of xt (F16 or BF16; BF16 is converted to fp16, exact for
  * 2^-14 <= |x| <= 65504), Y: device [M][n_out] of yt.  The weight enters the
- * tensor-core product as its fp16 dequantised value; accumulation is fp32.
+ * tensor-core product as its fp16 dequantised value (bit for bit what
+ * vqlin_dequant writes); accumulation is fp32.  For d = 8 layers with one
+ * codebook and no outlier block the weight tiles are dequantised in shared
+ * memory inside the GEMM, and the workspace only holds BF16 activations
+ * converted to fp16 (M * n_in * 2 bytes; unused for F16); other layers
+ * dequantise the whole weight into the workspace first.
  * workspace: device memory of at least vqlin_gemm_workspace_size(h, M) bytes,
  * 256-byte aligned, owned by the caller, not used concurrently by another call.
  * Errors additionally: WORKSPACE, UNSUPPORTED (M < 1 or n_in % 8 != 0).

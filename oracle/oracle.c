@@ -154,6 +154,8 @@ typedef struct {
   int32_t n_ocols; const int32_t* ocols;
   int32_t ko, bits_o; const uint16_t* cbo; const uint8_t* codes_o; int64_t stride_o;
   int64_t nnz; const int32_t* row_ptr; const int32_t* col_idx; const uint16_t* values;
+  int64_t vsr_nb; const int32_t* vsr_row_ptr; const int32_t* vsr_pos; const uint16_t* vsr_values;
+  int32_t n_groups; int32_t cb_symmetry;
 } oracle_layer;
 
 enum { ORACLE_OK = 0, ORACLE_BAD_INDEX = 1, ORACLE_BAD_VALUE = 2, ORACLE_BAD_CSR = 3, ORACLE_OOM = 4 };
@@ -172,16 +174,45 @@ static int column_ranks(const oracle_layer* L, uint8_t* is_out, int32_t* rank) {
   return ORACLE_OK;
 }
 
-/* Decoded indices of one weight element (i, j) that is not in the sparse set.
-   Returns the codebook pointers and entries through the out-arguments. */
+static int32_t n_main_cols(const oracle_layer* L) { return L->n_in - L->n_ocols; }
+static int32_t n_main_sub(const oracle_layer* L) { return (n_main_cols(L) + L->d - 1) / L->d; }
+static int32_t n_groups_of(const oracle_layer* L) { return L->n_groups > 1 ? L->n_groups : 1; }
+
+/* Codebook group of main sub-vector s (VPTQ page, "Outlier Elimination", on group partitioning:
+   independent codebooks per group; reading: contiguous ranges of ceil(n_sub / n_groups)
+   positions). */
+static int32_t group_of(const oracle_layer* L, int32_t s) {
+  const int32_t G = n_groups_of(L), n_sub = n_main_sub(L);
+  if (G == 1) return 0;
+  const int32_t size = (n_sub + G - 1) / G;
+  return s / size;
+}
+
+/* Element e (0..d-1) of entry i1 of group g's main codebook.  A symmetric codebook (SCVQ
+   summary: symmetry constraints shrink the codebook to a quarter) stores k1/4 base entries;
+   entry t*(k1/4) + b is base entry b under sign pattern t: 0 none, 1 all negated, 2 odd
+   elements negated, 3 even elements negated (fp16 negation flips the sign bit, exactly). */
+static uint16_t main_entry(const oracle_layer* L, int32_t g, uint32_t i1, int32_t e) {
+  const int32_t d = L->d;
+  if (!L->cb_symmetry) return L->cb1[((int64_t)g * L->k1 + i1) * d + e];
+  const uint32_t k1s = (uint32_t)L->k1 / 4u;
+  const uint32_t t = i1 / k1s, b = i1 % k1s;
+  const uint16_t v = L->cb1[((int64_t)g * k1s + b) * d + e];
+  const int neg = (t == 1) || (t == 2 && (e & 1)) || (t == 3 && !(e & 1));
+  return neg ? (uint16_t)(v ^ 0x8000u) : v;
+}
+
+/* Decoded codebook values of one weight element (i, j) that is not in the sparse set: the fp16
+   bits of the first-stage (or outlier-block) element in *h1, and a pointer to the residual
+   element in *e2 (NULL when there is none). */
 static int element_codes(const oracle_layer* L, const uint8_t* is_out, const int32_t* rank, int32_t i,
-                         int32_t j, const uint16_t** e1, const uint16_t** e2) {
+                         int32_t j, uint16_t* h1, const uint16_t** e2) {
   int32_t d = L->d;
   if (is_out[j]) {
     int32_t p = rank[j];
     uint32_t io = oracle_field(L->codes_o + (int64_t)i * L->stride_o, p / d, L->bits_o);
     if (io >= (uint32_t)L->ko) return ORACLE_BAD_INDEX;
-    *e1 = L->cbo + (int64_t)io * d + (p % d);
+    *h1 = *(L->cbo + (int64_t)io * d + (p % d));
     *e2 = NULL;                        /* the residual codebook does not apply */
   } else {
     int32_t q = rank[j];
@@ -189,14 +220,54 @@ static int element_codes(const oracle_layer* L, const uint8_t* is_out, const int
     uint32_t i1 = L->bits1 >= 32 ? f : (f & ((1u << L->bits1) - 1u));
     uint32_t i2 = L->bits2 ? (f >> L->bits1) : 0;
     if (i1 >= (uint32_t)L->k1) return ORACLE_BAD_INDEX;
-    *e1 = L->cb1 + (int64_t)i1 * d + (q % d);
+    const int32_t g = group_of(L, q / d);
+    *h1 = main_entry(L, g, i1, q % d);
     if (L->k2 > 0) {
       if (i2 >= (uint32_t)L->k2) return ORACLE_BAD_INDEX;
-      *e2 = L->cb2 + (int64_t)i2 * d + (q % d);
+      *e2 = L->cb2 + ((int64_t)g * L->k2 + i2) * d + (q % d);
     } else {
       *e2 = NULL;
     }
   }
+  return ORACLE_OK;
+}
+
+/* Main-column ids in order (main_col[q] = the q-th column that is not an outlier column). */
+static void main_columns(const oracle_layer* L, const uint8_t* is_out, int32_t* main_col) {
+  int32_t q = 0;
+  for (int32_t j = 0; j < L->n_in; ++j) if (!is_out[j]) main_col[q++] = j;
+}
+
+/* VSR blocks (SCVQ summary: a structured sparse format for salient weights that sit
+   contiguously within rows; reading: whole main-column sub-vectors, REPLACE): structure,
+   finiteness, and no element shared with the CSR matrix. */
+static int check_vsr(const oracle_layer* L, const uint8_t* is_out, const int32_t* rank) {
+  if (L->vsr_nb == 0) return ORACLE_OK;
+  const int32_t d = L->d, n_sub = n_main_sub(L);
+  if (L->vsr_row_ptr[0] != 0 || L->vsr_row_ptr[L->n_out] != L->vsr_nb) return ORACLE_BAD_CSR;
+  for (int32_t i = 0; i < L->n_out; ++i) {
+    if (L->vsr_row_ptr[i + 1] < L->vsr_row_ptr[i]) return ORACLE_BAD_CSR;
+    for (int32_t b = L->vsr_row_ptr[i]; b < L->vsr_row_ptr[i + 1]; ++b) {
+      const int32_t s = L->vsr_pos[b];
+      if (s < 0 || s >= n_sub || (b > L->vsr_row_ptr[i] && L->vsr_pos[b - 1] >= s)) return ORACLE_BAD_CSR;
+      for (int32_t t = 0; t < d; ++t)
+        if (((L->vsr_values[(int64_t)b * d + t] >> 10) & 0x1F) == 31) return ORACLE_BAD_VALUE;
+    }
+    if (L->nnz > 0)
+      for (int32_t e = L->row_ptr[i]; e < L->row_ptr[i + 1]; ++e) {
+        const int32_t j = L->col_idx[e];
+        if (is_out[j]) continue;
+        for (int32_t b = L->vsr_row_ptr[i]; b < L->vsr_row_ptr[i + 1]; ++b)
+          if (L->vsr_pos[b] == rank[j] / d) return ORACLE_BAD_CSR;   /* element in both */
+      }
+  }
+  return ORACLE_OK;
+}
+
+static int check_shape(const oracle_layer* L) {
+  const int32_t n_sub = n_main_sub(L);
+  if (L->n_groups < 0 || (n_sub > 0 && n_groups_of(L) > n_sub)) return ORACLE_BAD_VALUE;
+  if (L->cb_symmetry && (L->cb_symmetry != 1 || L->k1 % 4 != 0)) return ORACLE_BAD_VALUE;
   return ORACLE_OK;
 }
 
@@ -258,22 +329,33 @@ static int check_csr(const oracle_layer* L) {
 int oracle_dequant_exact(const oracle_layer* L, uint16_t* W, int64_t ldw) {
   uint8_t* is_out = (uint8_t*)malloc((size_t)L->n_in);
   int32_t* rank = (int32_t*)malloc(sizeof(int32_t) * (size_t)L->n_in);
-  int rc = (is_out && rank) ? ORACLE_OK : ORACLE_OOM;
+  int32_t* main_col = (int32_t*)malloc(sizeof(int32_t) * (size_t)L->n_in);
+  int rc = (is_out && rank && main_col) ? ORACLE_OK : ORACLE_OOM;
+  if (rc == ORACLE_OK) rc = check_shape(L);
   if (rc == ORACLE_OK) rc = column_ranks(L, is_out, rank);
   if (rc == ORACLE_OK) rc = check_csr(L);
+  if (rc == ORACLE_OK) rc = check_vsr(L, is_out, rank);
+  if (rc == ORACLE_OK) main_columns(L, is_out, main_col);
   for (int32_t i = 0; rc == ORACLE_OK && i < L->n_out; ++i) {
     const uint16_t* hr = L->rs ? &L->rs[i] : NULL;
     for (int32_t j = 0; rc == ORACLE_OK && j < L->n_in; ++j) {
-      const uint16_t *e1, *e2;
-      rc = element_codes(L, is_out, rank, i, j, &e1, &e2);
+      uint16_t h1;
+      const uint16_t* e2;
+      rc = element_codes(L, is_out, rank, i, j, &h1, &e2);
       if (rc != ORACLE_OK) break;
-      rc = exact_body_f16(*e1, e2, hr, L->cs ? &L->cs[j] : NULL, &W[(int64_t)i * ldw + j]);
+      rc = exact_body_f16(h1, e2, hr, L->cs ? &L->cs[j] : NULL, &W[(int64_t)i * ldw + j]);
     }
     if (rc == ORACLE_OK && L->nnz > 0)
       for (int32_t e = L->row_ptr[i]; e < L->row_ptr[i + 1]; ++e)
         W[(int64_t)i * ldw + L->col_idx[e]] = L->values[e];   /* REPLACE: exact outliers */
+    if (rc == ORACLE_OK && L->vsr_nb > 0)
+      for (int32_t b = L->vsr_row_ptr[i]; b < L->vsr_row_ptr[i + 1]; ++b)
+        for (int32_t t = 0; t < L->d; ++t) {
+          const int32_t q = L->vsr_pos[b] * L->d + t;
+          if (q < n_main_cols(L)) W[(int64_t)i * ldw + main_col[q]] = L->vsr_values[(int64_t)b * L->d + t];
+        }
   }
-  free(is_out); free(rank);
+  free(is_out); free(rank); free(main_col);
   return rc;
 }
 
@@ -281,17 +363,22 @@ int oracle_dequant_exact(const oracle_layer* L, uint16_t* W, int64_t ldw) {
 int oracle_dequant_f64_rows(const oracle_layer* L, const int32_t* rows, int32_t n_rows, double* W) {
   uint8_t* is_out = (uint8_t*)malloc((size_t)L->n_in);
   int32_t* rank = (int32_t*)malloc(sizeof(int32_t) * (size_t)L->n_in);
-  int rc = (is_out && rank) ? ORACLE_OK : ORACLE_OOM;
+  int32_t* main_col = (int32_t*)malloc(sizeof(int32_t) * (size_t)L->n_in);
+  int rc = (is_out && rank && main_col) ? ORACLE_OK : ORACLE_OOM;
+  if (rc == ORACLE_OK) rc = check_shape(L);
   if (rc == ORACLE_OK) rc = column_ranks(L, is_out, rank);
   if (rc == ORACLE_OK) rc = check_csr(L);
+  if (rc == ORACLE_OK) rc = check_vsr(L, is_out, rank);
+  if (rc == ORACLE_OK) main_columns(L, is_out, main_col);
   for (int32_t t = 0; rc == ORACLE_OK && t < n_rows; ++t) {
     int32_t i = rows[t];
     double r = L->rs ? oracle_f16_to_f64(L->rs[i]) : 1.0;
     for (int32_t j = 0; j < L->n_in; ++j) {
-      const uint16_t *e1, *e2;
-      rc = element_codes(L, is_out, rank, i, j, &e1, &e2);
+      uint16_t h1;
+      const uint16_t* e2;
+      rc = element_codes(L, is_out, rank, i, j, &h1, &e2);
       if (rc != ORACLE_OK) break;
-      double v = oracle_f16_to_f64(*e1);
+      double v = oracle_f16_to_f64(h1);
       if (e2) v = v + oracle_f16_to_f64(*e2);
       v = v * r;
       if (L->cs) v = v * oracle_f16_to_f64(L->cs[j]);
@@ -300,8 +387,14 @@ int oracle_dequant_f64_rows(const oracle_layer* L, const int32_t* rows, int32_t 
     if (rc == ORACLE_OK && L->nnz > 0)
       for (int32_t e = L->row_ptr[i]; e < L->row_ptr[i + 1]; ++e)
         W[(int64_t)t * L->n_in + L->col_idx[e]] = oracle_f16_to_f64(L->values[e]);
+    if (rc == ORACLE_OK && L->vsr_nb > 0)
+      for (int32_t b = L->vsr_row_ptr[i]; b < L->vsr_row_ptr[i + 1]; ++b)
+        for (int32_t u = 0; u < L->d; ++u) {
+          const int32_t q = L->vsr_pos[b] * L->d + u;
+          if (q < n_main_cols(L)) W[(int64_t)t * L->n_in + main_col[q]] = oracle_f16_to_f64(L->vsr_values[(int64_t)b * L->d + u]);
+        }
   }
-  free(is_out); free(rank);
+  free(is_out); free(rank); free(main_col);
   return rc;
 }
 

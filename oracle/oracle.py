@@ -49,6 +49,8 @@ class _Layer(C.Structure):
         ("ko", C.c_int32), ("bits_o", C.c_int32), ("cbo", C.c_void_p), ("codes_o", C.c_void_p),
         ("stride_o", C.c_int64),
         ("nnz", C.c_int64), ("row_ptr", C.c_void_p), ("col_idx", C.c_void_p), ("values", C.c_void_p),
+        ("vsr_nb", C.c_int64), ("vsr_row_ptr", C.c_void_p), ("vsr_pos", C.c_void_p), ("vsr_values", C.c_void_p),
+        ("n_groups", C.c_int32), ("cb_symmetry", C.c_int32),
     ]
 
 
@@ -119,8 +121,12 @@ def _marshal(layer):
     row_ptr = arr("row_ptr", np.int32)
     col_idx = arr("col_idx", np.int32)
     values = arr("values", np.uint16)
+    vsr_row_ptr = arr("vsr_row_ptr", np.int32)
+    vsr_pos = arr("vsr_pos", np.int32)
+    vsr_values = arr("vsr_values", np.uint16)
     n_ocols = 0 if ocols is None else int(ocols.size)
     nnz = 0 if col_idx is None else int(col_idx.size)
+    nvsr = 0 if vsr_pos is None else int(vsr_pos.size)
     L = _Layer(
         n_out=layer.n_out, n_in=layer.n_in, d=layer.d,
         k1=layer.k1, bits1=layer.bits1, k2=getattr(layer, "k2", 0) or 0, bits2=getattr(layer, "bits2", 0) or 0,
@@ -132,6 +138,9 @@ def _marshal(layer):
         stride_o=0 if codes_o is None else (codes_o.shape[1] if codes_o.ndim == 2 else codes_o.size // layer.n_out),
         nnz=nnz, row_ptr=_ptr(row_ptr) if nnz else None, col_idx=_ptr(col_idx) if nnz else None,
         values=_ptr(values) if nnz else None,
+        vsr_nb=nvsr, vsr_row_ptr=_ptr(vsr_row_ptr) if nvsr else None, vsr_pos=_ptr(vsr_pos) if nvsr else None,
+        vsr_values=_ptr(vsr_values) if nvsr else None,
+        n_groups=int(getattr(layer, "n_groups", 1) or 1), cb_symmetry=int(getattr(layer, "cb_symmetry", 0) or 0),
     )
     return L, keep
 

@@ -173,6 +173,22 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
   const int d = D->d, w = D->bits1 + D->bits2;
   const int32_t n_main = D->n_in - D->n_ocols;
   const int32_t n_sub = (int32_t)ceil_div(n_main, d);
+  // codebook groups and the symmetric codebook
+  const int32_t G = D->n_groups > 1 ? D->n_groups : 1;
+  if (D->n_groups < 0 || (G > 1 && G > n_sub)) {
+    set_error("n_groups = %d: need 0 or 1 <= n_groups <= n_sub = %d", D->n_groups, n_sub);
+    return VQLIN_ERR_INVALID_ARG;
+  }
+  if (D->cb_symmetry != 0 && (D->cb_symmetry != 1 || D->k1 % 4 != 0)) {
+    set_error("cb_symmetry must be 0, or 1 with k1 %% 4 == 0 (k1 = %d)", D->k1);
+    return VQLIN_ERR_INVALID_ARG;
+  }
+  const int32_t k1s = D->cb_symmetry ? D->k1 / 4 : D->k1;   // stored entries per group
+  const int32_t g_size = G > 1 ? (int32_t)ceil_div(n_sub, G) : (n_sub > 0 ? n_sub : 1);
+  if (D->vsr_nblocks < 0 || D->vsr_nblocks > (int64_t)D->n_out * n_sub || D->vsr_nblocks > 0x7FFFFFFFll) {
+    set_error("vsr_nblocks out of range");
+    return VQLIN_ERR_INVALID_ARG;
+  }
   const int32_t n_sub_o = (int32_t)ceil_div(D->n_ocols, d);
   const int64_t row_bytes = ceil_div((int64_t)n_sub * w, 8);
   const int64_t row_bytes_o = ceil_div((int64_t)n_sub_o * D->bits_o, 8);
@@ -188,11 +204,11 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
   int prev_dev = 0;
   cudaGetDevice(&prev_dev);
   // ---- bring everything to the host
-  std::vector<uint8_t> codes, cb1, cb2, cbo, codes_o, rs, cs, ocols, rp, ci, vals;
+  std::vector<uint8_t> codes, cb1, cb2, cbo, codes_o, rs, cs, ocols, rp, ci, vals, vrp, vpos, vvals;
   vqlin_status st = VQLIN_OK;
   if (n_sub > 0) st = fetch(D->codes, (size_t)D->row_stride_bytes * D->n_out, host, codes, "codes");
-  if (!st) st = fetch(D->codebook1, (size_t)D->k1 * d * 2, host, cb1, "codebook1");
-  if (!st && D->k2) st = fetch(D->codebook2, (size_t)D->k2 * d * 2, host, cb2, "codebook2");
+  if (!st) st = fetch(D->codebook1, (size_t)G * k1s * d * 2, host, cb1, "codebook1");
+  if (!st && D->k2) st = fetch(D->codebook2, (size_t)G * D->k2 * d * 2, host, cb2, "codebook2");
   if (!st && D->row_scale) st = fetch(D->row_scale, (size_t)D->n_out * 2, host, rs, "row_scale");
   if (!st && D->col_scale) st = fetch(D->col_scale, (size_t)D->n_in * 2, host, cs, "col_scale");
   if (!st && D->n_ocols) {
@@ -205,6 +221,11 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
     if (!st) st = fetch(D->col_idx, (size_t)D->nnz * 4, host, ci, "col_idx");
     if (!st) st = fetch(D->values, (size_t)D->nnz * 2, host, vals, "values");
   }
+  if (!st && D->vsr_nblocks) {
+    st = fetch(D->vsr_row_ptr, (size_t)(D->n_out + 1) * 4, host, vrp, "vsr_row_ptr");
+    if (!st) st = fetch(D->vsr_pos, (size_t)D->vsr_nblocks * 4, host, vpos, "vsr_pos");
+    if (!st) st = fetch(D->vsr_values, (size_t)D->vsr_nblocks * d * 2, host, vvals, "vsr_values");
+  }
   if (st) return st;
 
   // ---- validate values
@@ -213,9 +234,28 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
     for (size_t i = 0; i < v.size() / 2; ++i) if (!f16_finite(p[i])) return false;
     return true;
   };
-  if (!finite_all(cb1) || !finite_all(cb2) || !finite_all(cbo) || !finite_all(rs) || !finite_all(cs)) {
-    set_error("a codebook or scale entry is inf or NaN");
+  if (!finite_all(cb1) || !finite_all(cb2) || !finite_all(cbo) || !finite_all(rs) || !finite_all(cs) ||
+      !finite_all(vvals)) {
+    set_error("a codebook, scale or VSR entry is inf or NaN");
     return VQLIN_ERR_INVALID_DATA;
+  }
+  // A symmetric codebook holds k1/4 base entries per group; entry t * (k1/4) + b of the k1 that
+  // the indices address is base entry b under sign pattern t (0 none, 1 all elements negated, 2
+  // odd elements negated, 3 even elements negated).  Negating fp16 flips its sign bit, so the
+  // expansion is exact; every kernel then reads k1 entries per group.
+  if (D->cb_symmetry) {
+    std::vector<uint8_t> full((size_t)G * D->k1 * d * 2);
+    const uint16_t* base = as<uint16_t>(cb1);
+    uint16_t* out16 = reinterpret_cast<uint16_t*>(full.data());
+    for (int32_t g = 0; g < G; ++g)
+      for (int32_t t = 0; t < 4; ++t)
+        for (int32_t b = 0; b < k1s; ++b)
+          for (int e = 0; e < d; ++e) {
+            const bool neg = t == 1 || (t == 2 && (e & 1)) || (t == 3 && !(e & 1));
+            const uint16_t v = base[((size_t)g * k1s + b) * d + e];
+            out16[(((size_t)g * D->k1) + (size_t)t * k1s + b) * d + e] = neg ? (uint16_t)(v ^ 0x8000u) : v;
+          }
+    cb1.swap(full);
   }
   // column classification
   std::vector<int32_t> colmap;   // main ids then outlier ids
@@ -300,8 +340,9 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
         } else {
           int32_t q = rank[j];
           uint32_t f = host_field(codes.data() + (size_t)i * D->row_stride_bytes, q / d, w);
-          body = f16_val(C1[(size_t)(f & m1) * d + q % d]);
-          if (C2) body += f16_val(C2[(size_t)(f >> D->bits1) * d + q % d]);
+          const size_t g = (size_t)((q / d) / g_size);
+          body = f16_val(C1[(g * D->k1 + (f & m1)) * d + q % d]);
+          if (C2) body += f16_val(C2[(g * D->k2 + (f >> D->bits1)) * d + q % d]);
         }
         body *= ri;
         if (D->col_scale) body *= f16_val(as<uint16_t>(cs)[j]);
@@ -314,13 +355,67 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
     }
   }
 
-  // tensor-core decode layout (see vqlin_internal.cuh)
+  // VSR blocks: structure, no element shared with the CSR matrix, and the fused-product form
+  // delta = v - body per element (double, stored fp32; 0 past the last main column)
+  std::vector<float> vdelta((size_t)D->vsr_nblocks * d, 0.f);
+  if (D->vsr_nblocks) {
+    const int32_t* r = as<int32_t>(vrp);
+    const int32_t* ps = as<int32_t>(vpos);
+    const uint16_t* vv = as<uint16_t>(vvals);
+    const uint16_t* C1 = as<uint16_t>(cb1);
+    const uint16_t* C2 = D->k2 ? as<uint16_t>(cb2) : nullptr;
+    if (r[0] != 0 || r[D->n_out] != D->vsr_nblocks) { set_error("vsr_row_ptr must start at 0 and end at vsr_nblocks"); return VQLIN_ERR_INVALID_DATA; }
+    std::vector<int32_t> main_col(n_main);
+    for (int32_t j = 0; j < D->n_in; ++j) if (!is_out[j]) main_col[rank[j]] = j;
+    const int32_t* cr = D->nnz ? as<int32_t>(rp) : nullptr;
+    const int32_t* cc = D->nnz ? as<int32_t>(ci) : nullptr;
+    for (int32_t i = 0; i < D->n_out; ++i) {
+      if (r[i + 1] < r[i]) { set_error("vsr_row_ptr decreases at row %d", i); return VQLIN_ERR_INVALID_DATA; }
+      const double ri = D->row_scale ? f16_val(as<uint16_t>(rs)[i]) : 1.0;
+      int32_t e = cr ? cr[i] : 0;
+      const int32_t e_end = cr ? cr[i + 1] : 0;
+      for (int32_t b = r[i]; b < r[i + 1]; ++b) {
+        const int32_t sv = ps[b];
+        if (sv < 0 || sv >= n_sub || (b > r[i] && ps[b - 1] >= sv)) {
+          set_error("row %d: VSR positions must be strictly increasing and in [0, n_sub)", i);
+          return VQLIN_ERR_INVALID_DATA;
+        }
+        const uint32_t f = host_field(codes.data() + (size_t)i * D->row_stride_bytes, sv, w);
+        const size_t g = (size_t)(sv / g_size);
+        for (int t = 0; t < d; ++t) {
+          const int32_t q = sv * d + t;
+          if (q >= n_main) break;
+          const int32_t j = main_col[q];
+          while (e < e_end && cc[e] < j) ++e;           // CSR columns of the row, increasing
+          if (e < e_end && cc[e] == j) {
+            set_error("row %d column %d is in both the CSR matrix and a VSR block", i, j);
+            return VQLIN_ERR_INVALID_DATA;
+          }
+          double body = f16_val(C1[(g * D->k1 + (f & m1)) * d + t]);
+          if (C2) body += f16_val(C2[(g * D->k2 + (f >> D->bits1)) * d + t]);
+          body *= ri;
+          if (D->col_scale) body *= f16_val(as<uint16_t>(cs)[j]);
+          vdelta[(size_t)b * d + t] = (float)(f16_val(vv[(size_t)b * d + t]) - body);
+        }
+      }
+    }
+  }
+
+  // tensor-core decode layout (see vqlin_internal.cuh).  With codebook groups its fields hold
+  // g * k1 + i1 | (g * k2 + i2) << tc_b1, widened to the next width its kernels take.
   std::vector<uint8_t> tcodes;
   int32_t n_ls = 0;
   int64_t tstride = 0;
-  if (d == 8 && n_sub > 0 && (w == 8 || w == 12 || w == 16 || w == 24 || w == 32)) {
+  int tc_b1 = D->bits1, tc_w = w;
+  if (G > 1) {
+    auto bits_for = [](int64_t n) { int b = 1; while ((1ll << b) < n) ++b; return b; };
+    tc_b1 = bits_for((int64_t)G * D->k1);
+    const int need = tc_b1 + (D->k2 ? bits_for((int64_t)G * D->k2) : 0);
+    tc_w = need <= 8 ? 8 : need <= 12 ? 12 : need <= 16 ? 16 : need <= 24 ? 24 : need <= 32 ? 32 : 0;
+  }
+  if (d == 8 && n_sub > 0 && (tc_w == 8 || tc_w == 12 || tc_w == 16 || tc_w == 24 || tc_w == 32)) {
     n_ls = (int32_t)ceil_div(n_sub, 64);
-    tstride = (int64_t)n_ls * 8 * w;
+    tstride = (int64_t)n_ls * 8 * tc_w;
     const int64_t rows_pad = round_up(D->n_out, 16);
     tcodes.assign((size_t)(rows_pad * tstride), 0);
     for (int32_t i = 0; i < D->n_out; ++i) {
@@ -331,7 +426,12 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
           for (int ps = 0; ps < 16; ++ps) {
             int32_t sv = 64 * ls + 4 * ps + t;
             if (sv >= n_sub) continue;   // padding fields stay 0 (a valid index; x' is 0 there)
-            host_put_field(dst, (int64_t)ls * 64 + t * 16 + ps, w, host_field(row, sv, w));
+            uint32_t f = host_field(row, sv, w);
+            if (G > 1) {
+              const uint32_t g = (uint32_t)(sv / g_size);
+              f = (g * (uint32_t)D->k1 + (f & m1)) | ((D->k2 ? g * (uint32_t)D->k2 + (f >> D->bits1) : 0u) << tc_b1);
+            }
+            host_put_field(dst, (int64_t)ls * 64 + t * 16 + ps, tc_w, f);
           }
     }
   }
@@ -342,16 +442,18 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
   std::vector<uint16_t> cs_wpos;
   std::vector<float> cs_bound;
   int32_t cs_P = 0, cs_H = 0, cs_E = 0, cs_rpp = 0, cs_lbits = 0, cs_ebits = 0, cs_epw = 0;
-  if (d == 8 && D->k2 == 0 && D->k1 > 10240 && n_sub > 0 && n_sub <= 65536) {
+  // the codebook-stationary layout indexes the virtual codebook of all groups, g * k1 + i1
+  const int64_t kv = (int64_t)G * D->k1;
+  if (d == 8 && D->k2 == 0 && kv > 10240 && kv <= (1 << 24) && n_sub > 0 && n_sub <= 65536) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     auto bitlen = [](int64_t v) { int b = 0; while ((1ll << b) <= v) ++b; return b < 1 ? 1 : b; };
     const int H = D->n_out >= 2048 ? 2 : 1;
-    int P = (int)std::max<int64_t>(ceil_div(D->k1, 1023), std::max(1, sms / H));
-    P = std::min(P, D->k1);
-    const int E = (int)ceil_div(D->k1, P);
-    P = (int)ceil_div(D->k1, E);
+    int P = (int)std::max<int64_t>(ceil_div(kv, 1023), std::max(1, sms / H));
+    P = (int)std::min<int64_t>(P, kv);
+    const int E = (int)ceil_div(kv, P);
+    P = (int)ceil_div(kv, E);
     const int rpp = (int)ceil_div(D->n_out, H);
     const int lb = bitlen(E), rb = bitlen(rpp - 1), eb = lb + rb;   // local indices 0..E (E = null entry)
     const int epw = eb <= 21 ? 3 : (eb <= 32 ? 2 : 0);
@@ -370,7 +472,7 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
       };
       for (int32_t sv = 0; sv < n_sub; ++sv) {
         for (int32_t i = 0; i < D->n_out; ++i) {
-          uint32_t idx = host_field(codes.data() + (size_t)i * D->row_stride_bytes, sv, w) & m1;
+          uint32_t idx = (uint32_t)((sv / g_size) * D->k1) + (host_field(codes.data() + (size_t)i * D->row_stride_bytes, sv, w) & m1);
           const int pp = (int)(idx / (uint32_t)E), hh = i / rpp, cc = pp * H + hh;
           put(cc, ((uint32_t)(i - hh * rpp) << lb) | (idx - (uint32_t)pp * E), sv);
           per_row[(size_t)cc * rpp + (i - hh * rpp)] += 1;
@@ -383,7 +485,7 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
       // so a row's partial sum in the block stays below bound * max|x'|.
       const uint16_t* C1 = as<uint16_t>(cb1);
       std::vector<double> l1(P, 0.0);
-      for (int32_t k = 0; k < D->k1; ++k) {
+      for (int32_t k = 0; k < (int32_t)kv; ++k) {
         double a1 = 0;
         for (int t = 0; t < 8; ++t) a1 += std::fabs(f16_val(C1[(size_t)k * 8 + t]));
         l1[k / E] = std::max(l1[k / E], a1);
@@ -472,6 +574,9 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
   L.stride = stride; L.stride_o = D->n_ocols ? stride_o : 0;
   L.codes = up.put<uint8_t>(codes_r.data(), codes_r.size());
   L.codes_o = D->n_ocols ? up.put<uint8_t>(codes_o_r.data(), codes_o_r.size()) : nullptr;
+  L.n_groups = G;
+  L.g_size = g_size;
+  L.g_magic = g_size > 1 ? (uint32_t)(((1ull << 32) + (uint64_t)g_size - 1) / (uint64_t)g_size) : 0u;
   L.cb1 = up.put<__half>(cb1.data(), cb1.size());
   L.cb2 = D->k2 ? up.put<__half>(cb2.data(), cb2.size()) : nullptr;
   L.cbo = D->n_ocols ? up.put<__half>(cbo.data(), cbo.size()) : nullptr;
@@ -485,6 +590,13 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
     L.val = up.put<uint16_t>(vals.data(), vals.size());
     L.delta = up.put<float>(delta.data(), delta.size() * 4);
     L.col16 = col16.empty() ? nullptr : up.put<uint16_t>(col16.data(), col16.size() * 2);
+  }
+  L.vsr_nb = D->vsr_nblocks;
+  if (D->vsr_nblocks) {
+    L.vsr_rp = up.put<int32_t>(vrp.data(), vrp.size());
+    L.vsr_pos = up.put<int32_t>(vpos.data(), vpos.size());
+    L.vsr_val = up.put<uint16_t>(vvals.data(), vvals.size());
+    L.vsr_delta = up.put<float>(vdelta.data(), vdelta.size() * 4);
   }
   L.tcodes = tcodes.empty() ? nullptr : up.put<uint8_t>(tcodes.data(), tcodes.size());
   if (!cs_words.empty()) {
@@ -500,6 +612,8 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
   }
   L.n_ls = n_ls;
   L.tstride = tstride;
+  L.tc_w = tcodes.empty() ? 0 : tc_w;
+  L.tc_bits1 = tc_b1;
   L.tcodes_rows = tcodes.empty() ? 0 : (int32_t)round_up(D->n_out, 16);
   if (up.st == VQLIN_OK) up.st = cuda_status(cudaStreamSynchronize((cudaStream_t)stream), "create sync");
   if (up.st != VQLIN_OK) {
@@ -512,18 +626,21 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
   I.n_out = D->n_out; I.n_in = D->n_in; I.d = d; I.n_sub = n_sub; I.n_sub_o = n_sub_o; I.n_ocols = D->n_ocols;
   I.nnz = D->nnz;
   I.index_bytes = row_bytes * D->n_out + (D->n_ocols ? row_bytes_o * D->n_out : 0);
-  I.codebook_bytes = 2ll * d * (D->k1 + D->k2 + (D->n_ocols ? D->ko : 0));
+  I.codebook_bytes = 2ll * d * ((int64_t)G * (k1s + D->k2) + (D->n_ocols ? D->ko : 0));
   I.scale_bytes = (D->row_scale ? 2ll * D->n_out : 0) + (D->col_scale ? 2ll * D->n_in : 0);
   I.sparse_bytes = D->nnz ? D->nnz * 6 + 4ll * (D->n_out + 1) : 0;
+  I.vsr_bytes = D->vsr_nblocks ? D->vsr_nblocks * (4 + 2ll * d) + 4ll * (D->n_out + 1) : 0;
   {
-    // VPTQ "Compression ratio calculation": 16*M / (V*k*16 + M*ceil(log2 k)/V)
+    // VPTQ "Compression ratio calculation": 16*M / (V*k*16 + M*ceil(log2 k)/V), with the main
+    // codebooks counted as stored (n_groups of k1s entries)
     double M = (double)D->n_out * D->n_in;
     int lb = 0;
     while ((1ll << lb) < D->k1) ++lb;
-    double ratio = 16.0 * M / ((double)d * D->k1 * 16.0 + M * lb / d);
+    double ratio = 16.0 * M / ((double)d * G * k1s * 16.0 + M * lb / d);
     I.vptq_compression_ratio = ratio;
     I.vptq_bits_per_weight = 16.0 / ratio;
-    double total_bits = 8.0 * (I.index_bytes + I.codebook_bytes + I.scale_bytes + I.sparse_bytes + 4ll * D->n_ocols);
+    double total_bits = 8.0 * (I.index_bytes + I.codebook_bytes + I.scale_bytes + I.sparse_bytes + I.vsr_bytes +
+                               4ll * D->n_ocols);
     I.total_bits_per_weight = total_bits / M;
   }
   cudaSetDevice(prev_dev);
@@ -585,7 +702,9 @@ static size_t ws_align(size_t b) { return (b + 255) & ~size_t(255); }
 
 size_t vqlin_gemm_workspace_size(const vqlin_handle* h, int64_t M) {
   if (!h || M < 1) return 0;
-  size_t w = ws_align((size_t)h->L.n_out * h->L.n_in * 2);
+  // the fused path needs room only for bf16 activations converted to fp16; the two-phase path
+  // also holds the dequantised fp16 weight
+  size_t w = gemm_fused_supported(h->L) ? 0 : ws_align((size_t)h->L.n_out * h->L.n_in * 2);
   size_t x = ws_align((size_t)M * h->L.n_in * 2);
   return w + x;
 }
@@ -604,6 +723,18 @@ vqlin_status vqlin_gemm(const vqlin_handle* h, const void* X, vqlin_dtype xt, in
     return VQLIN_ERR_WORKSPACE;
   }
   cudaStream_t s = (cudaStream_t)stream;
+  if (gemm_fused_supported(h->L)) {
+    // weight tiles dequantised in shared memory inside the GEMM; bf16 activations are first
+    // converted to fp16 in the workspace (exact in the precondition's range)
+    const __half* A = reinterpret_cast<const __half*>(X);
+    if (xt == VQLIN_BF16) {
+      __half* X16 = reinterpret_cast<__half*>(workspace);
+      vqlin_status st = cuda_status(launch_convert_to_f16(X, xt, M * h->L.n_in, X16, s), "gemm convert launch");
+      if (st) return st;
+      A = X16;
+    }
+    return cuda_status(launch_gemm_vq(h->L, A, M, Y, yt, s), "gemm launch");
+  }
   __half* W = reinterpret_cast<__half*>(workspace);
   __half* X16 = reinterpret_cast<__half*>(reinterpret_cast<char*>(workspace) + ws_align((size_t)h->L.n_out * h->L.n_in * 2));
   vqlin_status st = cuda_status(launch_dequant(h->L, W, h->L.n_in, s), "gemm dequant launch");

@@ -57,8 +57,9 @@ __global__ void __launch_bounds__(256) k_dequant_body(Layer L, __half* __restric
     __half* Wrow = W + (int64_t)i * ldw;
     if (s < L.n_sub) {
       uint32_t f = read_field(L.codes + (int64_t)i * L.stride, s, L.w);
-      const __half* e1 = L.cb1 + (size_t)(f & m1) * D;
-      const __half* e2 = L.cb2 ? L.cb2 + (size_t)(f >> L.bits1) * D : nullptr;
+      const size_t g = (size_t)group_of(L, s);        // codebook group of position s
+      const __half* e1 = L.cb1 + (g * L.k1 + (f & m1)) * D;
+      const __half* e2 = L.cb2 ? L.cb2 + (g * L.k2 + (f >> L.bits1)) * D : nullptr;
       int q0 = s * D;
       unsigned short outv[D];
 #pragma unroll
@@ -119,6 +120,20 @@ __global__ void k_dequant_sparse(Layer L, __half* __restrict__ W, int64_t ldw) {
   }
 }
 
+// VSR blocks REPLACE whole sub-vectors bit for bit.  One warp per row, lanes over its blocks.
+__global__ void k_dequant_vsr(Layer L, __half* __restrict__ W, int64_t ldw) {
+  const int warps = (blockDim.x >> 5) * gridDim.x;
+  for (int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < L.n_out; i += warps) {
+    for (int b = L.vsr_rp[i] + (threadIdx.x & 31); b < L.vsr_rp[i + 1]; b += 32) {
+      const int q0 = L.vsr_pos[b] * L.d;
+      for (int t = 0; t < L.d && q0 + t < L.n_main; ++t) {
+        const int j = L.colmap ? L.colmap[q0 + t] : q0 + t;
+        W[(int64_t)i * ldw + j] = __ushort_as_half(L.vsr_val[(int64_t)b * L.d + t]);
+      }
+    }
+  }
+}
+
 __global__ void k_convert_f16(const unsigned short* __restrict__ X, vqlin_dtype xt, int64_t n,
                               __half* __restrict__ out) {
   int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -171,7 +186,7 @@ __global__ void __launch_bounds__(512, 1) k_dequant_cs(Layer L, __half* __restri
   const int p = c / H, h = c - p * H;
   const int row0 = h * RPP;
   const int nrows = min(RPP, L.n_out - row0);
-  const int slice0 = p * E, E_p = max(0, min(E, L.k1 - slice0));
+  const int slice0 = p * E, E_p = max(0, min(E, L.n_groups * L.k1 - slice0));   // virtual codebook of all groups
   uint4* cbs = reinterpret_cast<uint4*>(smem);                                        // [E + 1][8]
   float* cf = reinterpret_cast<float*>(smem + (size_t)(E + 1) * COPIES * 16);         // [n_sub * 8]
   float* rf = cf + (size_t)L.n_sub * 8;                                               // [RPP]
@@ -271,6 +286,12 @@ cudaError_t launch_dequant(const Layer& L, __half* W, int64_t ldw, cudaStream_t 
   if (L.nnz > 0) {
     note_launches(1);
     k_dequant_sparse<<<grid_for((int64_t)L.n_out * 32, 256), 256, 0, s>>>(L, W, ldw);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (L.vsr_nb > 0) {
+    note_launches(1);
+    k_dequant_vsr<<<grid_for((int64_t)L.n_out * 32, 256), 256, 0, s>>>(L, W, ldw);
     return cudaGetLastError();
   }
   return cudaSuccess;

@@ -76,16 +76,15 @@ __global__ void __launch_bounds__(kThreads) k_gemv_generic(Layer L, const void* 
   extern __shared__ __align__(16) unsigned char smem[];
   float* xs = reinterpret_cast<float*>(smem);                       // [NB][chunk]
   __half* cb1s = reinterpret_cast<__half*>(xs + NB * chunk);
-  __half* cb2s = cb1s + (size_t)L.k1 * D;
-  __half* cbos = cb2s + (size_t)L.k2 * D;
+  __half* cb2s = cb1s + (size_t)L.n_groups * L.k1 * D;
+  __half* cbos = cb2s + (size_t)L.n_groups * L.k2 * D;
   const __half* cb1 = L.cb1;
   const __half* cb2 = L.cb2;
   const __half* cbo = L.cbo;
   if (CB_SMEM) {
-    const int n16 = ((L.k1 + L.k2 + L.ko) * D * 2) / 16;   // all three are whole multiples of 4 bytes
     const uint4* srcs[3] = {reinterpret_cast<const uint4*>(L.cb1), reinterpret_cast<const uint4*>(L.cb2),
                             reinterpret_cast<const uint4*>(L.cbo)};
-    int lens[3] = {L.k1 * D * 2, L.k2 * D * 2, L.ko * D * 2};
+    int lens[3] = {L.n_groups * L.k1 * D * 2, L.n_groups * L.k2 * D * 2, L.ko * D * 2};   // whole 4-byte units
     unsigned char* dst = reinterpret_cast<unsigned char*>(cb1s);
     for (int part = 0; part < 3; ++part) {
       // copy in 4-byte units (an entry is 2*d bytes, d even), eight loads in flight per thread
@@ -102,7 +101,6 @@ __global__ void __launch_bounds__(kThreads) k_gemv_generic(Layer L, const void* 
       }
       dst += lens[part];
     }
-    (void)n16;
     cb1 = cb1s; cb2 = L.cb2 ? cb2s : nullptr; cbo = cbos;
   }
   pdl_wait();      // x and y belong to the previous grid until it completes
@@ -152,11 +150,14 @@ __global__ void __launch_bounds__(kThreads) k_gemv_generic(Layer L, const void* 
           const int s = sb + 32 * u;
           if (s >= s1) break;
           const uint32_t f = fs[u];
+          const int g = group_of(L, s);
           float c[D];
-          if (CB_SMEM) load_centroid_smem<D>(cb1, f & m1, c); else load_centroid<D>(cb1, f & m1, c);
+          const uint32_t e1 = (uint32_t)g * L.k1 + (f & m1);
+          if (CB_SMEM) load_centroid_smem<D>(cb1, e1, c); else load_centroid<D>(cb1, e1, c);
           if (cb2) {
             float c2[D];
-            if (CB_SMEM) load_centroid_smem<D>(cb2, f >> L.bits1, c2); else load_centroid<D>(cb2, f >> L.bits1, c2);
+            const uint32_t e2 = (uint32_t)g * L.k2 + (f >> L.bits1);
+            if (CB_SMEM) load_centroid_smem<D>(cb2, e2, c2); else load_centroid<D>(cb2, e2, c2);
 #pragma unroll
             for (int k = 0; k < D; ++k) c[k] += c2[k];
           }
@@ -202,6 +203,7 @@ __global__ void __launch_bounds__(kThreads) k_gemv_generic(Layer L, const void* 
 #pragma unroll
     for (int b = 0; b < NB; ++b) sp[b] = 0.f;
     if (L.nnz > 0) sparse_row_terms<NB>(L, x, xt, batch, row, lane, 32, sp);
+    if (L.vsr_nb > 0) vsr_row_terms<NB>(L, x, xt, batch, row, lane, 32, sp);
     const float rsc = L.rs ? __half2float(L.rs[row]) : 1.f;
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
@@ -223,7 +225,7 @@ static cudaError_t launch_generic_nb(const Layer& L, const void* x, vqlin_dtype 
   int need_o = L.n_sub_o * D;
   if (need_o > chunk) chunk = ((need_o + 32 * D - 1) / (32 * D)) * (32 * D);
   size_t xs_bytes = (size_t)NB * chunk * 4;
-  size_t cb_bytes = (size_t)(L.k1 + L.k2 + L.ko) * D * 2;
+  size_t cb_bytes = ((size_t)L.n_groups * (L.k1 + L.k2) + L.ko) * D * 2;
   bool cb_smem = xs_bytes + cb_bytes <= 200 * 1024;
   size_t smem = xs_bytes + (cb_smem ? cb_bytes : 0);
   dim3 grid((L.n_out + kRowsPerCta - 1) / kRowsPerCta);

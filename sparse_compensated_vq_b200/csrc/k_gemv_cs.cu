@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_cs(Args a) {
   const int p = c / H, h = c - p * H;
   const int row0 = h * RPP;
   const int nrows = min(RPP, L.n_out - row0);
-  const int slice0 = p * E, E_p = max(0, min(E, L.k1 - slice0));
+  const int slice0 = p * E, E_p = max(0, min(E, L.n_groups * L.k1 - slice0));   // virtual codebook of all groups
   const int n_sub = L.n_sub;
   const int B = a.batch;
   const Carve cv(E, n_sub, NB, RPP, COPIES);
@@ -393,6 +393,19 @@ __global__ void __launch_bounds__(256) k_cs_finalize(Layer L, const float* __res
         }
       }
     }
+    // VSR blocks of the same four rows (lanes over each row's blocks)
+    if (L.vsr_nb > 0) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int64_t row = ib + q;
+        float tv[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) tv[b] = 0.f;
+        if (row < L.n_out) vsr_row_terms<NB>(L, x, xt, batch, row, lane, 32, tv);
+#pragma unroll
+        for (int b = 0; b < NB; ++b) sp[q][b] += tv[b];
+      }
+    }
 #pragma unroll
     for (int q = 0; q < 4; ++q)
 #pragma unroll
@@ -544,7 +557,7 @@ cudaError_t launch_gemv_cs(const Layer& L, const void* x, vqlin_dtype xt, int ba
   // shared memory requested, the word buffer must hold whole 32-word groups, every slot's local
   // index and row must fit the slice and the row half, and the partial planes must fit the
   // workspace.  A plan that fails any of them is refused instead of launched.
-  if (smem > smem_max || a.words_cap % 32 != 0 || (int64_t)L.cs_P * L.cs_E < L.k1 ||
+  if (smem > smem_max || a.words_cap % 32 != 0 || (int64_t)L.cs_P * L.cs_E < (int64_t)L.n_groups * L.k1 ||
       (int64_t)L.cs_H * L.cs_rpp < L.n_out || (1ll << L.cs_local_bits) <= L.cs_E ||
       (size_t)(L.cs_E + 1) * copies * 16 > cv.xs || (size_t)L.cs_P * batch * L.n_out * 4 > ws_bytes) {
     set_error("codebook-stationary decode: inconsistent launch plan (refused)");

@@ -103,6 +103,9 @@ struct Args {
   int n_chunks;       // ceil(n_kslabs / ks)
   int xs_cols;        // columns of x' held in shared memory (chunk columns, or all)
   int xs_all;         // 1: x' for all main columns staged once per CTA
+  // warp-task kernel: the main columns split into wt_nch chunks of wt_cs kernel slabs; block b
+  // serves chunk b / wt_bpc (staging its x' once) and a task is one row tile over wt_spt slabs
+  int wt_cs, wt_nch, wt_bpc, wt_spt;
 };
 
 template <int NT, int W, bool CB_SMEM, int COPIES>
@@ -116,8 +119,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
   // ---- shared memory carve-up
   unsigned char* sp = smem;
   uint4* cb1s = reinterpret_cast<uint4*>(sp);
-  uint4* cb2s = cb1s + (CB_SMEM ? (size_t)L.k1 * COPIES : 0);
-  sp = reinterpret_cast<unsigned char*>(cb2s + (CB_SMEM ? (size_t)L.k2 * COPIES : 0));
+  uint4* cb2s = cb1s + (CB_SMEM ? (size_t)L.n_groups * L.k1 * COPIES : 0);
+  sp = reinterpret_cast<unsigned char*>(cb2s + (CB_SMEM ? (size_t)L.n_groups * L.k2 * COPIES : 0));
   __half* xh = reinterpret_cast<__half*>(sp);                      // [batch][xs_cols]
   __half* xl = xh + (size_t)a.batch * a.xs_cols;
   float* red = reinterpret_cast<float*>(xl + (size_t)a.batch * a.xs_cols);   // [rtt][16][8*NT]
@@ -126,15 +129,15 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int B = a.batch;
-  const uint32_t m1 = (1u << L.bits1) - 1u;
+  const uint32_t m1 = (1u << L.tc_bits1) - 1u;   // first-stage bits of the tensor-core layout
 
   // ---- codebooks into shared memory (COPIES interleaved copies: entry k of copy c at k*COPIES + c)
   if (CB_SMEM) {
     const uint4* c1 = reinterpret_cast<const uint4*>(L.cb1);
-    for (int i = threadIdx.x; i < L.k1 * COPIES; i += THREADS) cb1s[i] = __ldg(c1 + i / COPIES);
+    for (int i = threadIdx.x; i < L.n_groups * L.k1 * COPIES; i += THREADS) cb1s[i] = __ldg(c1 + i / COPIES);
     if (L.k2) {
       const uint4* c2 = reinterpret_cast<const uint4*>(L.cb2);
-      for (int i = threadIdx.x; i < L.k2 * COPIES; i += THREADS) cb2s[i] = __ldg(c2 + i / COPIES);
+      for (int i = threadIdx.x; i < L.n_groups * L.k2 * COPIES; i += THREADS) cb2s[i] = __ldg(c2 + i / COPIES);
     }
   }
   // ---- layer-only prefetch for this block's first task, before the wait: the index words of
@@ -263,6 +266,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
     for (int b = 0; b < BP; ++b) { spv[b] = task == task0 ? spv0[b] : 0.f; ov[b] = 0.f; }
     if (first_chunk && row_ok) {
       if (L.nnz > 0 && task != task0) sparse_row_terms<BP>(L, a.x, a.xt, B, row, sub, lanes_per_row, spv);
+      if (L.vsr_nb > 0) vsr_row_terms<BP>(L, a.x, a.xt, B, row, sub, lanes_per_row, spv);
       for (int s = sub; s < L.n_sub_o; s += lanes_per_row) {
         uint32_t f = read_field(L.codes_o + row * L.stride_o, s, L.bits_o);
         uint4 u = __ldg(reinterpret_cast<const uint4*>(L.cbo) + f);
@@ -334,6 +338,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
 #pragma unroll
         for (int j = 0; j < G; ++j) {
           const uint32_t f0 = field_of<W>(w0, p0 + j), f1 = field_of<W>(w1, p0 + j);
+          // tensor-core layout fields already hold g * k + i for codebook group g
           if (CB_SMEM) {
             c0[j] = cb1s[(f0 & m1) * COPIES + (lane & (COPIES - 1))];
             c1[j] = cb1s[(f1 & m1) * COPIES + (lane & (COPIES - 1))];
@@ -343,11 +348,11 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
           }
           if (L.k2) {
             if (CB_SMEM) {
-              e0[j] = cb2s[(f0 >> L.bits1) * COPIES + (lane & (COPIES - 1))];
-              e1[j] = cb2s[(f1 >> L.bits1) * COPIES + (lane & (COPIES - 1))];
+              e0[j] = cb2s[(f0 >> L.tc_bits1) * COPIES + (lane & (COPIES - 1))];
+              e1[j] = cb2s[(f1 >> L.tc_bits1) * COPIES + (lane & (COPIES - 1))];
             } else {
-              e0[j] = __ldg(reinterpret_cast<const uint4*>(L.cb2) + (f0 >> L.bits1));
-              e1[j] = __ldg(reinterpret_cast<const uint4*>(L.cb2) + (f1 >> L.bits1));
+              e0[j] = __ldg(reinterpret_cast<const uint4*>(L.cb2) + (f0 >> L.tc_bits1));
+              e1[j] = __ldg(reinterpret_cast<const uint4*>(L.cb2) + (f1 >> L.tc_bits1));
             }
           }
         }
@@ -437,21 +442,21 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) k_gemv_wt(Args a) {
   const Layer& L = a.L;
   extern __shared__ __align__(16) unsigned char smem[];
   uint4* cb1s = reinterpret_cast<uint4*>(smem);
-  uint4* cb2s = cb1s + (CB_SMEM ? (size_t)L.k1 * COPIES : 0);
-  __half* xh = reinterpret_cast<__half*>(cb2s + (CB_SMEM ? (size_t)L.k2 * COPIES : 0));   // [batch][xs_cols]
+  uint4* cb2s = cb1s + (CB_SMEM ? (size_t)L.n_groups * L.k1 * COPIES : 0);
+  __half* xh = reinterpret_cast<__half*>(cb2s + (CB_SMEM ? (size_t)L.n_groups * L.k2 * COPIES : 0));   // [batch][xs_cols]
   __half* xl = xh + (size_t)a.batch * a.xs_cols;
   float* xo = reinterpret_cast<float*>(xl + (size_t)a.batch * a.xs_cols);               // [BP][n_sub_o*8]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int B = a.batch;
-  const uint32_t m1 = (1u << L.bits1) - 1u;
+  const uint32_t m1 = (1u << L.tc_bits1) - 1u;   // first-stage bits of the tensor-core layout
 
   if (CB_SMEM) {
     const uint4* c1 = reinterpret_cast<const uint4*>(L.cb1);
-    for (int i = threadIdx.x; i < L.k1 * COPIES; i += WT_THREADS) cb1s[i] = __ldg(c1 + i / COPIES);
+    for (int i = threadIdx.x; i < L.n_groups * L.k1 * COPIES; i += WT_THREADS) cb1s[i] = __ldg(c1 + i / COPIES);
     if (L.k2) {
       const uint4* c2 = reinterpret_cast<const uint4*>(L.cb2);
-      for (int i = threadIdx.x; i < L.k2 * COPIES; i += WT_THREADS) cb2s[i] = __ldg(c2 + i / COPIES);
+      for (int i = threadIdx.x; i < L.n_groups * L.k2 * COPIES; i += WT_THREADS) cb2s[i] = __ldg(c2 + i / COPIES);
     }
   }
   // x (and the accumulator) belong to the previous grid until it completes
@@ -468,21 +473,26 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) k_gemv_wt(Args a) {
     }
     xo[i] = v;
   }
-  // x' hi/lo for every main column, eight columns per thread, loads first
+  // this block's column chunk: kernel slabs [ks_beg, ks_end), main columns from col0
+  const int ch = blockIdx.x / a.wt_bpc, jb = blockIdx.x - ch * a.wt_bpc;
+  const int ks_beg = ch * a.wt_cs, ks_end = min(ks_beg + a.wt_cs, a.n_kslabs);
+  const int col0 = ks_beg * KSV * 8;
+  // x' hi/lo for the chunk's main columns, eight columns per thread, loads first
   {
     const int groups = a.xs_cols / 8;
     for (int i = threadIdx.x; i < B * groups; i += WT_THREADS) {
       const int b = i / groups, q = (i - b * groups) * 8;
+      const int qq = col0 + q;                         // main-column index of this group
       float v[8];
-      if (!L.colmap && a.xt != VQLIN_F32 && q + 8 <= L.n_main && (L.n_in & 7) == 0) {
+      if (!L.colmap && a.xt != VQLIN_F32 && qq + 8 <= L.n_main && (L.n_in & 7) == 0) {
         uint4 u = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const unsigned short*>(a.x) +
-                                                        (int64_t)b * L.n_in + q));
+                                                        (int64_t)b * L.n_in + qq));
         const unsigned short* hs = reinterpret_cast<const unsigned short*>(&u);
 #pragma unroll
         for (int k = 0; k < 8; ++k)
           v[k] = a.xt == VQLIN_F16 ? __half2float(__ushort_as_half(hs[k])) : __bfloat162float(__ushort_as_bfloat16(hs[k]));
         if (L.cs) {
-          uint4 cu = __ldg(reinterpret_cast<const uint4*>(L.cs + q));
+          uint4 cu = __ldg(reinterpret_cast<const uint4*>(L.cs + qq));
           const __half* cv = reinterpret_cast<const __half*>(&cu);
 #pragma unroll
           for (int k = 0; k < 8; ++k) v[k] *= __half2float(cv[k]);
@@ -490,7 +500,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) k_gemv_wt(Args a) {
       } else {
         int jj[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) jj[k] = q + k < L.n_main ? (L.colmap ? L.colmap[q + k] : q + k) : -1;
+        for (int k = 0; k < 8; ++k) jj[k] = qq + k < L.n_main ? (L.colmap ? L.colmap[qq + k] : qq + k) : -1;
 #pragma unroll
         for (int k = 0; k < 8; ++k) v[k] = jj[k] >= 0 ? load_as_float(a.x, a.xt, (int64_t)b * L.n_in + jj[k]) : 0.f;
         if (L.cs) {
@@ -513,12 +523,18 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) k_gemv_wt(Args a) {
   __syncthreads();
 
   const int n_rt = (L.n_out + 15) / 16;
-  const bool has_side = L.nnz > 0 || L.n_ocols > 0;
+  const bool has_side = L.nnz > 0 || L.n_ocols > 0 || L.vsr_nb > 0;
   const int n_side = has_side ? (L.n_out + 7) / 8 : 0;      // sparse / outlier tasks of 8 rows
-  const int n_main = n_rt * a.n_kslabs;
-  const int total = n_side + n_main;
-  for (int task = blockIdx.x * NW + warp; task < total; task += gridDim.x * NW) {
-    if (task < n_side) {
+  const int gpc = (ks_end - ks_beg + a.wt_spt - 1) / a.wt_spt;   // slab groups of this chunk
+  const int n_mt = n_rt * gpc;                                    // this chunk's MMA tasks
+  // the sparse / outlier tasks first (spread over every block), then this chunk's MMA tasks
+  // (spread over the chunk's blocks)
+  const int side_beg = blockIdx.x * NW + warp, side_step = gridDim.x * NW;
+  const int n_side_mine = side_beg < n_side ? (n_side - side_beg + side_step - 1) / side_step : 0;
+  const int total = n_side_mine + (jb * NW + warp < n_mt ? (n_mt - jb * NW - warp + a.wt_bpc * NW - 1) / (a.wt_bpc * NW) : 0);
+  for (int it = 0; it < total; ++it) {
+    const int task = it < n_side_mine ? side_beg + it * side_step : -1;
+    if (task >= 0) {
       // ---- fused sparse correction and outlier block for rows 8*task .. +8 (4 lanes per row)
       const int64_t row = (int64_t)task * 8 + (lane >> 2);
       const int sub = lane & 3;
@@ -527,6 +543,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) k_gemv_wt(Args a) {
 #pragma unroll
       for (int b = 0; b < BP; ++b) spv[b] = ov[b] = 0.f;
       if (ok && L.nnz > 0) sparse_row_terms<BP>(L, a.x, a.xt, B, row, sub, 4, spv);
+      if (ok && L.vsr_nb > 0) vsr_row_terms<BP>(L, a.x, a.xt, B, row, sub, 4, spv);
       if (ok) {
         for (int so = sub; so < L.n_sub_o; so += 4) {
           uint32_t f = read_field(L.codes_o + row * L.stride_o, so, L.bits_o);
@@ -555,17 +572,12 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) k_gemv_wt(Args a) {
       }
       continue;
     }
-    // ---- MMA task: row tile rt, kernel slab ks
-    const int mt = task - n_side;
-    const int rt = mt / a.n_kslabs, kslab = mt - rt * a.n_kslabs;
-    const int ls = kslab / NT, part = kslab - ls * NT;
+    // ---- MMA task: row tile rt over the kernel slabs of slab group sg of this chunk
+    const int mt = jb * NW + warp + (it - n_side_mine) * a.wt_bpc * NW;
+    const int rt = mt / gpc, sg = mt - rt * gpc;
+    const int kb0 = ks_beg + sg * a.wt_spt, kb1 = min(kb0 + a.wt_spt, ks_end);
     const int64_t R0 = (int64_t)rt * 16 + g;
     constexpr int NWORDS = (2 * W / NT + 3) / 4 + 1;
-    uint32_t w0[NWORDS], w1[NWORDS];
-    w0[NWORDS - 1] = w1[NWORDS - 1] = 0;
-    const uint8_t* blk0 = L.tcodes + R0 * L.tstride + (int64_t)ls * (8 * W) + t * (2 * W) + part * PS * W / 8;
-    load_sub<W, NT>(blk0, w0);
-    load_sub<W, NT>(blk0 + 8 * L.tstride, w1);
     const float r0 = (L.rs && R0 < L.n_out) ? __half2float(L.rs[R0]) : 1.f;
     const float r1 = (L.rs && R0 + 8 < L.n_out) ? __half2float(L.rs[R0 + 8]) : 1.f;
     // ACC independent accumulator sets, so consecutive MMAs do not wait on each other
@@ -574,7 +586,14 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) k_gemv_wt(Args a) {
     for (int q = 0; q < ACC; ++q)
 #pragma unroll
       for (int n = 0; n < NT; ++n) dacc[q][n][0] = dacc[q][n][1] = dacc[q][n][2] = dacc[q][n][3] = 0.f;
-    const int col_base = kslab * KSV * 8;
+    for (int kslab = kb0; kslab < kb1; ++kslab) {
+    const int ls = kslab / NT, part = kslab - ls * NT;
+    uint32_t w0[NWORDS], w1[NWORDS];
+    w0[NWORDS - 1] = w1[NWORDS - 1] = 0;
+    const uint8_t* blk0 = L.tcodes + R0 * L.tstride + (int64_t)ls * (8 * W) + t * (2 * W) + part * PS * W / 8;
+    load_sub<W, NT>(blk0, w0);
+    load_sub<W, NT>(blk0 + 8 * L.tstride, w1);
+    const int col_base = (kslab - ks_beg) * KSV * 8;   // inside the staged chunk
     // gathers per batch: never more than the slab's pair-steps (PS is 4 when NT = 4)
     constexpr int G = ((W >= 24) ? 4 : 8) < PS ? ((W >= 24) ? 4 : 8) : PS;
     static_assert(PS % G == 0, "pair-step batches must tile the kernel slab");
@@ -584,6 +603,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) k_gemv_wt(Args a) {
 #pragma unroll
       for (int j = 0; j < G; ++j) {
         const uint32_t f0 = field_of<W>(w0, p0 + j), f1 = field_of<W>(w1, p0 + j);
+        // tensor-core layout fields already hold g * k + i for codebook group g
         if (CB_SMEM) {
           c0[j] = cb1s[(f0 & m1) * COPIES + (lane & (COPIES - 1))];
           c1[j] = cb1s[(f1 & m1) * COPIES + (lane & (COPIES - 1))];
@@ -593,11 +613,11 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) k_gemv_wt(Args a) {
         }
         if (L.k2) {
           if (CB_SMEM) {
-            e0[j] = cb2s[(f0 >> L.bits1) * COPIES + (lane & (COPIES - 1))];
-            e1[j] = cb2s[(f1 >> L.bits1) * COPIES + (lane & (COPIES - 1))];
+            e0[j] = cb2s[(f0 >> L.tc_bits1) * COPIES + (lane & (COPIES - 1))];
+            e1[j] = cb2s[(f1 >> L.tc_bits1) * COPIES + (lane & (COPIES - 1))];
           } else {
-            e0[j] = __ldg(reinterpret_cast<const uint4*>(L.cb2) + (f0 >> L.bits1));
-            e1[j] = __ldg(reinterpret_cast<const uint4*>(L.cb2) + (f1 >> L.bits1));
+            e0[j] = __ldg(reinterpret_cast<const uint4*>(L.cb2) + (f0 >> L.tc_bits1));
+            e1[j] = __ldg(reinterpret_cast<const uint4*>(L.cb2) + (f1 >> L.tc_bits1));
           }
         }
       }
@@ -621,6 +641,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) k_gemv_wt(Args a) {
         }
       }
     }
+    }  // kernel slabs of the task
     float d[NT][4];
 #pragma unroll
     for (int n = 0; n < NT; ++n)
@@ -681,7 +702,7 @@ static cudaError_t launch_wt_w(const Args& args, bool cb_smem, int copies, size_
 
 template <int NT>
 static cudaError_t launch_wt_nt(const Args& args, bool cb_smem, int copies, size_t smem, int grid, cudaStream_t s) {
-  switch (args.L.w) {
+  switch (args.L.tc_w) {
     case 8: return launch_wt_w<NT, 8>(args, cb_smem, copies, smem, grid, s);
     case 12: return launch_wt_w<NT, 12>(args, cb_smem, copies, smem, grid, s);
     case 16: return launch_wt_w<NT, 16>(args, cb_smem, copies, smem, grid, s);
@@ -718,7 +739,7 @@ static cudaError_t launch_w(const Args& args, bool cb_smem, int copies, size_t s
 
 template <int NT>
 static cudaError_t launch_nt(const Args& args, bool cb_smem, int copies, size_t smem, int grid, cudaStream_t s) {
-  switch (args.L.w) {
+  switch (args.L.tc_w) {
     case 8: return launch_w<NT, 8>(args, cb_smem, copies, smem, grid, s);
     case 12: return launch_w<NT, 12>(args, cb_smem, copies, smem, grid, s);
     case 16: return launch_w<NT, 16>(args, cb_smem, copies, smem, grid, s);
@@ -735,7 +756,8 @@ static size_t gemv_acc_bytes(const Layer& L, int batch) {
 }
 
 bool tc_supported(const Layer& L) {
-  return L.d == 8 && L.tcodes != nullptr && (L.w == 8 || L.w == 12 || L.w == 16 || L.w == 24 || L.w == 32);
+  return L.d == 8 && L.tcodes != nullptr &&
+         (L.tc_w == 8 || L.tc_w == 12 || L.tc_w == 16 || L.tc_w == 24 || L.tc_w == 32);
 }
 
 size_t gemv_workspace_bytes(const Layer& L, int batch) {
@@ -769,9 +791,10 @@ cudaError_t launch_gemv_tc(const Layer& L, const void* x, vqlin_dtype xt, int ba
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const size_t smem_max = 227 * 1024;
   // codebooks: as many interleaved copies (<= 8) as fit next to x'
-  const size_t cb_entries = (size_t)L.k1 + L.k2;
+  const size_t cb_entries = (size_t)L.n_groups * ((size_t)L.k1 + L.k2);
   Args a;
   a.L = L; a.x = x; a.xt = xt; a.batch = batch; a.y = y; a.yt = yt; a.acc = nullptr;
+  a.wt_cs = 0; a.wt_nch = 1; a.wt_bpc = 1; a.wt_spt = 1;   // set by the warp-task plan below
   a.n_kslabs = (L.n_sub + KSV - 1) / KSV;
   a.ks = a.n_kslabs < WARPS ? a.n_kslabs : WARPS;
   // round ks down to a divisor of WARPS so that rtt * ks == WARPS when several row tiles share a CTA
@@ -814,24 +837,61 @@ cudaError_t launch_gemv_tc(const Layer& L, const void* x, vqlin_dtype xt, int ba
     float* acc = nullptr;
     if (yt == VQLIN_F32) acc = reinterpret_cast<float*>(y);
     else if (ws && ws_bytes >= acc_bytes) acc = reinterpret_cast<float*>(ws);
+    // x' for every column next to the codebooks (as many interleaved copies as fit) when that
+    // fits; otherwise the columns are split into chunks of whole kernel slabs, each staged once
+    // by the blocks that serve it
     int wcopies = 0;
     bool wcb = false;
+    int cs = a.n_kslabs;                              // kernel slabs per chunk
+    const size_t slab_x = (size_t)batch * KSV * 8 * 4;   // x' (hi + lo fp16) of one kernel slab
     for (int c = 8; c >= 1; c >>= 1) {
       if (cb_entries * 16 * c <= 160 * 1024 && cb_entries * 16 * c + x_all + xo_bytes + 256 <= smem_max) {
         wcopies = c; wcb = true; break;
       }
     }
-    const size_t wsmem = (wcb ? cb_entries * 16 * wcopies : 0) + x_all + xo_bytes + 64;
-    if (acc && wsmem <= smem_max) {
+    if (!wcb) {
+      int fit = 0;
+      for (int c = 8; c >= 1; c >>= 1) {
+        const size_t cbb = cb_entries * 16 * c;
+        if (cbb > 160 * 1024 || cbb + xo_bytes + 256 + slab_x > smem_max) continue;
+        fit = (int)((smem_max - cbb - xo_bytes - 256) / slab_x);
+        if (c == 1 || fit >= 4) { wcopies = c; wcb = true; break; }
+      }
+      if (!wcb) fit = (int)((smem_max - xo_bytes - 256) / slab_x);   // codebook gathered from L2
+      cs = fit < a.n_kslabs ? fit : a.n_kslabs;
+    }
+    const int nch = cs > 0 ? (a.n_kslabs + cs - 1) / cs : 0;
+    const size_t wsmem = (wcb ? cb_entries * 16 * wcopies : 0) + (size_t)batch * cs * KSV * 8 * 4 + xo_bytes + 64;
+    if (acc && cs > 0 && wsmem <= smem_max) {
       Args w = a;
       w.acc = acc;
       w.xs_all = 1;
-      w.xs_cols = all_cols;
-      const int n_side = (L.nnz > 0 || L.n_ocols > 0) ? (L.n_out + 7) / 8 : 0;
-      const int total = n_side + n_rt * a.n_kslabs;
+      w.xs_cols = cs * KSV * 8;
+      const int n_side = (L.nnz > 0 || L.n_ocols > 0 || L.vsr_nb > 0) ? (L.n_out + 7) / 8 : 0;
       const int per_sm = (int)(smem_max / (wsmem + 1024)) >= 2 ? 2 : 1;
-      int grid = sms * per_sm;
-      if (grid > (total + WARPS - 1) / WARPS) grid = (total + WARPS - 1) / WARPS;
+      const int nw = per_sm == 2 ? 8 : 16;             // warps per block (launch_wt_cfg's choice)
+      int grid, bpc, spt = 1;
+      if (nch == 1) {
+        const int total = n_side + n_rt * a.n_kslabs;
+        grid = sms * per_sm;
+        if (grid > (total + WARPS - 1) / WARPS) grid = (total + WARPS - 1) / WARPS;
+        bpc = grid;
+      } else {
+        bpc = sms * per_sm / nch;
+        if (bpc < 1) bpc = 1;
+        grid = nch * bpc;
+        // a task covers spt slabs of one row tile: about three tasks per warp
+        const int64_t slab_tasks = (int64_t)n_rt * a.n_kslabs, target = 3ll * grid * nw;
+        spt = (int)((slab_tasks + target - 1) / target);
+        if (spt > cs) spt = cs;
+        if (spt < 1) spt = 1;
+      }
+      w.wt_cs = cs; w.wt_nch = nch; w.wt_bpc = bpc; w.wt_spt = spt;
+      // plan checks: every chunk's slabs are staged, and the grid is whole chunks of blocks
+      if (grid != nch * bpc || (int64_t)nch * cs < a.n_kslabs || w.xs_cols < cs * KSV * 8) {
+        set_error("warp-task decode: inconsistent launch plan (refused)");
+        return cudaErrorInvalidConfiguration;
+      }
       cudaError_t e = launch_pdl(k_zero, dim3(small_grid((int64_t)batch * L.n_out)), 256, 0, s, acc,
                                  (int64_t)batch * L.n_out);
       if (e != cudaSuccess) return e;

@@ -28,19 +28,36 @@ struct Layer {
   const __half* rs;                     // [n_out] or null (= 1)
   const __half* cs;                     // [n_in]  or null (= 1)
   const int32_t* colmap;                // [n_in]: main column ids (q order) then outlier ids (p order); null if no outliers
+  // Codebook groups: main sub-vector position s decodes with codebook s / g_size (cb1 holds
+  // n_groups * k1 entries, cb2 n_groups * k2).  A symmetric codebook is expanded at create time
+  // into its k1 entries per group, so the kernels index cb1 the same way.
+  int32_t n_groups, g_size;
+  uint32_t g_magic;                     // ceil(2^32 / g_size): s / g_size = umulhi(s, g_magic) for s < 65536
   int64_t nnz;
   const int32_t* row_ptr;               // [n_out+1] (null if nnz == 0)
   const int32_t* col;                   // [nnz]
   const uint16_t* val;                  // [nnz] fp16 bits (exact replacement values)
   const float* delta;                   // [nnz] v - body, for the fused products
   const uint16_t* col16;                // [nnz] column ids as u16 when n_in <= 65536, else null
+  // VSR blocks (whole main-column sub-vectors, REPLACE): block b of row i is sub-vector
+  // vsr_pos[b], b in [vsr_rp[i], vsr_rp[i+1]); vsr_val its fp16 values [nb][d]; vsr_delta the
+  // fused-product form v - decoded body [nb][d] (fp32, 0 past the last main column)
+  int64_t vsr_nb;
+  const int32_t* vsr_rp;
+  const int32_t* vsr_pos;
+  const uint16_t* vsr_val;
+  const float* vsr_delta;
   // Tensor-core decode layout (d = 8, w in {8,12,16,24,32}; null otherwise): rows padded
   // to a multiple of 16; per row and per slab of 64 sub-vectors, for t = 0..3 the 16
   // fields of sub-vectors 64*slab + 4*ps + t (ps = 0..15), packed LSB-first.
+  // With codebook groups the fields of this layout hold g * k1 + i1 (and g * k2 + i2 above
+  // tc_bits1), widened to tc_w bits, so these kernels index the concatenated codebooks directly;
+  // with one group tc_w = w and tc_bits1 = bits1.
   const uint8_t* tcodes;
+  int32_t tc_w, tc_bits1;
   int32_t n_ls;                         // layout slabs per row
   int32_t tcodes_rows;                  // rows allocated in tcodes (n_out rounded up to 16)
-  int64_t tstride;                      // bytes per row = n_ls * 8 * w
+  int64_t tstride;                      // bytes per row = n_ls * 8 * tc_w
   // Codebook-stationary layout (large single-stage codebooks, d = 8; null otherwise):
   // block c = p * cs_H + h owns codebook slice p (entries [p*cs_E, (p+1)*cs_E), cs_E < 1024)
   // and row half h (rows [h*cs_rpp, ...)); its entries (row - h*cs_rpp) << cs_local_bits |
@@ -84,6 +101,10 @@ cudaError_t launch_gemv_cs(const Layer& L, const void* x, vqlin_dtype xt, int ba
                            void* ws, size_t ws_bytes, cudaStream_t s, bool* handled);
 cudaError_t launch_gemm_f16(const __half* A, const __half* W, int64_t M, int N, int K, void* Y, vqlin_dtype yt,
                             cudaStream_t s);
+// Fused prefill: weight tiles dequantised in shared memory and fed to the tensor cores
+// (d = 8, one codebook, no outlier block, n_in % 8 == 0).  X is fp16 [M][n_in], 16-byte aligned.
+bool gemm_fused_supported(const Layer& L);
+cudaError_t launch_gemm_vq(const Layer& L, const __half* X, int64_t M, void* Y, vqlin_dtype yt, cudaStream_t s);
 
 // ---- small device helpers shared by the library's kernels -----------------
 __device__ __forceinline__ float load_as_float(const void* p, vqlin_dtype t, int64_t i) {
@@ -232,6 +253,58 @@ __device__ __forceinline__ void sparse_finish(const Layer& L, const void* x, vql
   });
 }
 
+// Codebook group of main sub-vector position s (0 with one codebook).  Layout padding past the
+// last position (the tensor-core layout rounds positions up to whole slabs; their x' is 0) is
+// clamped to the last group, so every index stays inside the codebooks.
+__device__ __forceinline__ int group_of(const Layer& L, int s) {
+  if (L.n_groups <= 1) return 0;
+  const int g = L.g_size == 1 ? s : (s < 65536 ? (int)__umulhi((uint32_t)s, L.g_magic) : s / L.g_size);
+  return g < L.n_groups ? g : L.n_groups - 1;
+}
+
+// VSR term of one row, sum over its blocks b (sub, sub + stride, ...) of sum_t delta[b][t] *
+// x[batch][main column s*d + t]: the fused form of the block REPLACE (the caller reduces over its
+// `stride` lanes).
+template <int BP>
+__device__ __forceinline__ void vsr_row_terms(const Layer& L, const void* x, vqlin_dtype xt, int B, int64_t row,
+                                              int sub, int stride, float* spv) {
+  const int b_beg = L.vsr_rp[row], b_end = L.vsr_rp[row + 1];
+  const int d = L.d;
+  with_dtype(xt, [&](auto tag) {
+    constexpr int XT = decltype(tag)::value;
+    for (int b = b_beg + sub; b < b_end; b += stride) {
+      const int q0 = L.vsr_pos[b] * d;
+      const float* dl = L.vsr_delta + (int64_t)b * d;
+      if (XT != VQLIN_F32 && d == 8 && !L.colmap && q0 + 8 <= L.n_main && (L.n_in & 7) == 0) {
+        const float4 d0 = __ldg(reinterpret_cast<const float4*>(dl)), d1 = __ldg(reinterpret_cast<const float4*>(dl) + 1);
+        const float dv[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+#pragma unroll
+        for (int bb = 0; bb < BP; ++bb)
+          if (bb < B) {
+            const uint4 u = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const unsigned short*>(x) +
+                                                                (int64_t)bb * L.n_in + q0));
+            const unsigned short* hs = reinterpret_cast<const unsigned short*>(&u);
+            float a = spv[bb];
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+              a = fmaf(dv[t], XT == VQLIN_F16 ? __half2float(__ushort_as_half(hs[t])) : __bfloat162float(__ushort_as_bfloat16(hs[t])), a);
+            spv[bb] = a;
+          }
+      } else {
+        for (int t = 0; t < d; ++t) {
+          const int q = q0 + t;
+          if (q >= L.n_main) break;
+          const int j = L.colmap ? L.colmap[q] : q;
+          const float dv = dl[t];
+#pragma unroll
+          for (int bb = 0; bb < BP; ++bb)
+            if (bb < B) spv[bb] = fmaf(dv, ldx<XT>(x, (int64_t)bb * L.n_in + j), spv[bb]);
+        }
+      }
+    }
+  });
+}
+
 // Programmatic dependent launch.  Decode kernels are launched so that they may start
 // while the previous grid on the stream is still running; everything they do before
 // pdl_wait() reads only the layer (immutable after create) and writes only shared memory.
@@ -266,6 +339,6 @@ struct vqlin_handle {
   // info
   vqlin_info info;
   // allocations to free
-  void* allocs[24];
+  void* allocs[32];
   int n_allocs;
 };

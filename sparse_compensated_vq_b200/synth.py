@@ -20,6 +20,13 @@ SmolLM2-1.7B layers at 2-4 bits per weight; seeds PCG64(20260000 + n)):
   5 vlen      4096x4096 at vector length d in {4, 6, 8, 12} with a K=4096 fp16 codebook
               (12-bit codes: 3, 2, 1.5, 1 bits/weight), row+col scales, 1% uniform
               outliers: VPTQ's vector-length trend (one seed per d)
+  7 qproj_sym the qproj shape with a symmetric codebook: 16384 stored entries addressed as
+              65536 (SCVQ's quarter-size codebook)
+  8 smollm_vsr the seven SmolLM2-1.7B linears with their 2% salient weights stored as whole
+              sub-vectors (VSR blocks, 2% of the sub-vectors, position probability ~ |z|^4)
+              instead of scattered CSR entries
+  9 qproj_groups the qproj shape with its 512 positions split into 4 groups of 65536-entry
+              codebooks (VPTQ's group_num)
 """
 from __future__ import annotations
 
@@ -111,6 +118,12 @@ class LayerData:
     row_ptr: Optional[np.ndarray] = None  # int32 [n_out+1]
     col_idx: Optional[np.ndarray] = None  # int32 [nnz]
     values: Optional[np.ndarray] = None   # uint16 fp16 [nnz]
+    # VSR blocks: whole main-column sub-vectors replaced (block-row format)
+    vsr_row_ptr: Optional[np.ndarray] = None  # int32 [n_out+1]
+    vsr_pos: Optional[np.ndarray] = None      # int32 [nblocks]
+    vsr_values: Optional[np.ndarray] = None   # uint16 fp16 [nblocks, d]
+    n_groups: int = 1                         # codebook groups over the sub-vector positions
+    cb_symmetry: int = 0                      # 1: codebook1 stores k1/4 base entries (sign patterns)
     name: str = ""
     # the decoded fields the generator drew (for tests of the packer only)
     fields: Optional[np.ndarray] = None
@@ -132,18 +145,25 @@ class LayerData:
     def nnz(self) -> int:
         return 0 if self.col_idx is None else int(self.col_idx.size)
 
+    @property
+    def vsr_nblocks(self) -> int:
+        return 0 if self.vsr_pos is None else int(self.vsr_pos.size)
+
     def abi_bytes(self) -> dict:
         """Bytes of the stored layer in the description's own format (rows unpadded)."""
         w = self.bits1 + self.bits2
         idx = self.n_out * packed_row_bytes(self.n_sub, w)
         if self.n_ocols:
             idx += self.n_out * packed_row_bytes(self.n_sub_o, self.bits_o)
-        cb = 2 * self.d * (self.k1 + self.k2 + (self.ko if self.n_ocols else 0))
+        g = max(1, self.n_groups)
+        k1s = self.k1 // 4 if self.cb_symmetry else self.k1
+        cb = 2 * self.d * (g * (k1s + self.k2) + (self.ko if self.n_ocols else 0))
         sc = (2 * self.n_out if self.row_scale is not None else 0) + (2 * self.n_in if self.col_scale is not None else 0)
         sp = self.nnz * 6 + (4 * (self.n_out + 1) if self.nnz else 0)
+        vs = self.vsr_nblocks * (4 + 2 * self.d) + (4 * (self.n_out + 1) if self.vsr_nblocks else 0)
         oc = 4 * self.n_ocols
-        return {"index": idx, "codebook": cb, "scale": sc, "sparse": sp, "ocols": oc,
-                "total": idx + cb + sc + sp + oc}
+        return {"index": idx, "codebook": cb, "scale": sc, "sparse": sp, "vsr": vs, "ocols": oc,
+                "total": idx + cb + sc + sp + vs + oc}
 
 
 def csr_from_positions(n_out: int, rows: np.ndarray, cols: np.ndarray, vals: np.ndarray):
@@ -185,13 +205,32 @@ def hessian_positions(rng, n_out: int, n_in: int, nnz: int):
     return np.concatenate(rows).astype(np.int64), np.concatenate(cols).astype(np.int64)
 
 
+def vsr_positions(rng, n_out: int, n_sub: int, nblocks: int, positions: str = "uniform"):
+    """(row, sub-vector) pairs of whole-sub-vector blocks: uniform over the grid, or with the
+    sub-vector position drawn with probability ~ |z_s|^4 (z ~ N(0,1)) and the rows uniform
+    without replacement within a position (salient input features, as for the Hessian-style
+    element outliers)."""
+    if positions == "uniform":
+        lin = rng.choice(n_out * n_sub, size=nblocks, replace=False)
+        return (lin // n_sub).astype(np.int64), (lin % n_sub).astype(np.int64)
+    return hessian_positions(rng, n_out, n_sub, nblocks)
+
+
 def random_layer(rng, n_out, n_in, d, k1, bits1, *, k2=0, bits2=0, cb_std=0.02, res_std=0.005,
                  row_scale=True, col_scale=False, n_ocols=0, ko=256, bits_o=8,
                  outlier_frac=0.01, outlier_scale=0.1, positions="uniform", nnz=None,
-                 stride=None, name="") -> LayerData:
-    """One layer with the given shape; every draw comes from `rng` in a fixed order."""
-    cb1 = f16_bits(rng.normal(0.0, cb_std, size=(k1, d)))
-    cb2 = f16_bits(rng.normal(0.0, res_std, size=(k2, d))) if k2 else None
+                 stride=None, name="", n_groups=1, cb_symmetry=0, vsr_frac=0.0, vsr_blocks=None,
+                 vsr_positions_kind="uniform") -> LayerData:
+    """One layer with the given shape; every draw comes from `rng` in a fixed order.
+
+    n_groups > 1 or cb_symmetry = 1 change the codebook draws (n_groups codebooks back to back;
+    k1/4 base entries each); VSR blocks (vsr_frac of the main sub-vectors, or vsr_blocks of them)
+    are drawn after everything else, and CSR entries that fall inside a block are dropped."""
+    g = max(1, n_groups)
+    k1s = k1 // 4 if cb_symmetry else k1
+    assert not cb_symmetry or k1 % 4 == 0
+    cb1 = f16_bits(rng.normal(0.0, cb_std, size=(g * k1s, d)))
+    cb2 = f16_bits(rng.normal(0.0, res_std, size=(g * k2, d))) if k2 else None
     ocols = np.sort(rng.choice(n_in, size=n_ocols, replace=False)).astype(np.int32) if n_ocols else np.zeros(0, np.int32)
     n_sub = -(-(n_in - n_ocols) // d)
     i1 = rng.integers(0, k1, size=(n_out, n_sub), dtype=np.int64)
@@ -219,11 +258,33 @@ def random_layer(rng, n_out, n_in, d, k1, bits1, *, k2=0, bits2=0, cb_std=0.02, 
         row_ptr, col_idx, values = csr_from_positions(n_out, rows, cols, vals)
     else:
         row_ptr = col_idx = values = None
+    vsr_rp = vsr_pos = vsr_vals = None
+    nb = vsr_blocks if vsr_blocks is not None else int(round(vsr_frac * n_out * n_sub))
+    if nb:
+        vr, vs = vsr_positions(rng, n_out, n_sub, nb, vsr_positions_kind)
+        vv = f16_bits(rng.standard_t(3, size=(nb, d)) * outlier_scale)
+        order = np.lexsort((vs, vr))
+        vr, vs, vv = vr[order], vs[order], vv[order]
+        vsr_rp = np.zeros(n_out + 1, dtype=np.int64)
+        np.cumsum(np.bincount(vr, minlength=n_out), out=vsr_rp[1:])
+        vsr_rp, vsr_pos, vsr_vals = vsr_rp.astype(np.int32), vs.astype(np.int32), vv
+        if row_ptr is not None:
+            # keep the element CSR disjoint from the blocks (main columns only carry blocks)
+            is_out = np.zeros(n_in, bool)
+            is_out[ocols] = True
+            qrank = np.cumsum(~is_out) - 1
+            blocked = set(zip(vr.tolist(), vs.tolist()))
+            rows_e = np.repeat(np.arange(n_out), np.diff(row_ptr))
+            keep = np.array([is_out[j] or (int(i), int(qrank[j]) // d) not in blocked
+                             for i, j in zip(rows_e, col_idx)], dtype=bool)
+            row_ptr, col_idx, values = csr_from_positions(n_out, rows_e[keep], col_idx[keep].astype(np.int64),
+                                                          values[keep])
     return LayerData(n_out=n_out, n_in=n_in, d=d, k1=k1, bits1=bits1, codes=codes, codebook1=cb1,
                      k2=k2, bits2=bits2, codebook2=cb2, row_scale=rs, col_scale=cs, ocols=ocols,
                      ko=ko if n_ocols else 0, bits_o=bits_o if n_ocols else 0, codebook_o=cbo,
                      codes_o=codes_o, row_ptr=row_ptr, col_idx=col_idx, values=values, name=name,
-                     fields=fields, fields_o=fields_o)
+                     fields=fields, fields_o=fields_o, vsr_row_ptr=vsr_rp, vsr_pos=vsr_pos, vsr_values=vsr_vals,
+                     n_groups=g, cb_symmetry=cb_symmetry)
 
 
 def activations(rng, batch: int, n_in: int, dtype: str = "f16") -> np.ndarray:
@@ -294,4 +355,33 @@ def vlen(d: int, batch: int = 1):
     rng = rng_for(5 * 100 + d)
     L = random_layer(rng, 4096, 4096, d, 4096, 12, cb_std=0.02, row_scale=True, col_scale=True,
                      outlier_frac=0.01, outlier_scale=0.1, name="vlen_4096x4096_d%d_k4096" % d)
+    return L, activations(rng, batch, 4096, "f16")
+
+
+def qproj_sym(batch: int = 1):
+    rng = rng_for(7)
+    L = random_layer(rng, 4096, 4096, 8, 65536, 16, cb_std=0.02, row_scale=True, col_scale=True,
+                     outlier_frac=0.01, outlier_scale=0.1, cb_symmetry=1,
+                     name="llama2_7b_qproj_4096x4096_d8_k65536_symmetric")
+    return L, activations(rng, batch, 4096, "f16")
+
+
+def smollm_vsr(batch: int = 1):
+    rng = rng_for(8)
+    layers, xs = [], []
+    for name, n_out, n_in in SMOLLM_SHAPES:
+        L = random_layer(rng, n_out, n_in, 8, 256, 8, cb_std=0.02, row_scale=True, col_scale=False,
+                         nnz=0, outlier_scale=0.1, vsr_frac=0.02, vsr_positions_kind="hessian",
+                         name="smollm2_1.7b_" + name + "_vsr")
+        layers.append(L)
+    for name, n_out, n_in in SMOLLM_SHAPES:
+        xs.append(activations(rng, batch, n_in, "bf16"))
+    return layers, xs
+
+
+def qproj_groups(batch: int = 1, groups: int = 4):
+    rng = rng_for(9)
+    L = random_layer(rng, 4096, 4096, 8, 65536, 16, cb_std=0.02, row_scale=True, col_scale=True,
+                     outlier_frac=0.01, outlier_scale=0.1, n_groups=groups,
+                     name="llama2_7b_qproj_4096x4096_d8_k65536_groups%d" % groups)
     return L, activations(rng, batch, 4096, "f16")

@@ -41,6 +41,9 @@ class vqlin_desc(C.Structure):
         ("ko", C.c_int32), ("bits_o", C.c_int32), ("codebook_o", C.c_void_p), ("codes_o", C.c_void_p),
         ("o_row_stride_bytes", C.c_int64),
         ("nnz", C.c_int64), ("row_ptr", C.c_void_p), ("col_idx", C.c_void_p), ("values", C.c_void_p),
+        ("vsr_nblocks", C.c_int64), ("vsr_row_ptr", C.c_void_p), ("vsr_pos", C.c_void_p),
+        ("vsr_values", C.c_void_p),
+        ("n_groups", C.c_int32), ("cb_symmetry", C.c_int32),
     ]
 
 
@@ -51,7 +54,7 @@ class vqlin_info(C.Structure):
         ("nnz", C.c_int64), ("index_bytes", C.c_int64), ("codebook_bytes", C.c_int64),
         ("scale_bytes", C.c_int64), ("sparse_bytes", C.c_int64),
         ("vptq_compression_ratio", C.c_double), ("vptq_bits_per_weight", C.c_double),
-        ("total_bits_per_weight", C.c_double),
+        ("total_bits_per_weight", C.c_double), ("vsr_bytes", C.c_int64),
     ]
 
 
@@ -172,6 +175,14 @@ def make_desc(layer, keep: list) -> vqlin_desc:
     D.nnz = nnz
     if nnz:
         D.row_ptr, D.col_idx, D.values = _ptr(arr("row_ptr", np.int32)), _ptr(col_idx), _ptr(arr("values", np.uint16))
+    vsr_pos = arr("vsr_pos", np.int32)
+    nb = 0 if vsr_pos is None else int(vsr_pos.size if on_host else vsr_pos.numel())
+    D.vsr_nblocks = nb
+    if nb:
+        D.vsr_row_ptr, D.vsr_pos = _ptr(arr("vsr_row_ptr", np.int32)), _ptr(vsr_pos)
+        D.vsr_values = _ptr(arr("vsr_values", np.uint16))
+    D.n_groups = int(getattr(layer, "n_groups", 1) or 1)
+    D.cb_symmetry = int(getattr(layer, "cb_symmetry", 0) or 0)
     return D
 
 

@@ -65,6 +65,31 @@ def exact_layer(L):
         for i in range(n_out):
             for e in range(int(L.row_ptr[i]), int(L.row_ptr[i + 1])):
                 csr[(i, int(L.col_idx[e]))] = int(L.values[e])
+    # VSR blocks: whole main-column sub-vectors, every element replaced
+    n_sub = -(-len(main) // d)
+    if getattr(L, "vsr_pos", None) is not None:
+        for i in range(n_out):
+            for b in range(int(L.vsr_row_ptr[i]), int(L.vsr_row_ptr[i + 1])):
+                s = int(L.vsr_pos[b])
+                for t in range(d):
+                    if s * d + t < len(main):
+                        j = main[s * d + t]
+                        assert (i, j) not in csr
+                        csr[(i, j)] = int(L.vsr_values[b, t])
+    groups = max(1, int(getattr(L, "n_groups", 1) or 1))
+    gsize = -(-n_sub // groups) if n_sub else 1
+    sym = int(getattr(L, "cb_symmetry", 0) or 0)
+
+    def main_value(g, i1, t):
+        """Element t of entry i1 of group g's main codebook (symmetric: base entry times a sign pattern)."""
+        if not sym:
+            return int(L.codebook1[g * L.k1 + i1, t])
+        k1s = L.k1 // 4
+        pattern, base = divmod(i1, k1s)
+        v = int(L.codebook1[g * k1s + base, t])
+        negate = pattern == 1 or (pattern == 2 and t % 2 == 1) or (pattern == 3 and t % 2 == 0)
+        return v ^ 0x8000 if negate else v
+
     W = [[None] * n_in for _ in range(n_out)]
     B = [[0] * n_in for _ in range(n_out)]
     for i in range(n_out):
@@ -86,10 +111,11 @@ def exact_layer(L):
                 f = field(row, q // d, w)
                 i1, i2 = f & ((1 << L.bits1) - 1), f >> L.bits1
                 assert i1 < L.k1
-                terms = [int(L.codebook1[i1, q % d])]
+                g = (q // d) // gsize
+                terms = [main_value(g, i1, q % d)]
                 if L.k2:
                     assert i2 < L.k2
-                    terms.append(int(L.codebook2[i2, q % d]))
+                    terms.append(int(L.codebook2[g * L.k2 + i2, q % d]))
             val = sum((f16_frac(t) for t in terms), Fraction(0))
             fl = np.float64(f16_float(terms[0]))
             for t in terms[1:]:

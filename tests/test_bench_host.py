@@ -11,7 +11,8 @@ import bench  # noqa: E402
 
 
 @pytest.mark.parametrize("name,batch", [("tiny", 1), ("qproj", 1), ("qproj", 4), ("downproj", 1), ("smollm", 1),
-                                        ("vlen4", 1), ("vlen6", 1), ("vlen8", 1), ("vlen12", 1)])
+                                        ("vlen4", 1), ("vlen6", 1), ("vlen8", 1), ("vlen12", 1), ("qproj_sym", 1),
+                                        ("qproj_groups", 1), ("smollm_vsr", 1)])
 def test_workloads_build(name, batch):
     wl = bench.make_workload(name, batch)
     assert wl.kind == "gemv"
@@ -25,6 +26,21 @@ def test_qproj_bytes_match_the_survey_count():
     # + fp16 row and column scales + fp16 x and y
     wl = bench.make_workload("qproj", 1)
     assert wl.bytes_per_step() == 6298668
+
+
+def test_vsr_and_symmetric_workloads_store_fewer_bytes():
+    """The VSR workload keeps its 2% salient weights as whole sub-vectors: 20 bytes per block of 8
+    against 48 for the same eight elements in CSR; the symmetric codebook stores a quarter of the
+    entries."""
+    vs = bench.make_workload("smollm_vsr", 1)
+    nb = sum(L.vsr_nblocks for L in vs.layers)
+    assert nb > 0 and all(L.nnz == 0 for L in vs.layers)
+    vsr_bytes = sum(L.abi_bytes()["vsr"] for L in vs.layers)
+    csr_bytes = sum(8 * L.vsr_nblocks * 6 + 4 * (L.n_out + 1) for L in vs.layers)
+    assert vsr_bytes < 0.45 * csr_bytes
+    q = bench.make_workload("qproj", 1).layers[0]
+    qs = bench.make_workload("qproj_sym", 1).layers[0]
+    assert qs.abi_bytes()["codebook"] * 4 == q.abi_bytes()["codebook"]
 
 
 def test_unknown_config_is_rejected():

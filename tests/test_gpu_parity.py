@@ -47,6 +47,16 @@ def small_layers():
         dict(n_out=40, n_in=192, d=12, k1=512, bits1=9, col_scale=True, nnz=30),
         # residual codebook + outlier block with n_in % 8 == 0, so the prefill GEMM covers both
         dict(n_out=96, n_in=208, d=4, k1=100, bits1=7, k2=30, bits2=5, col_scale=True, nnz=60, n_ocols=6, ko=50, bits_o=6),
+        # VSR blocks (SCVQ), codebook groups (VPTQ group_num), symmetric codebooks (SCVQ)
+        dict(n_out=130, n_in=264, d=8, k1=256, bits1=8, col_scale=True, nnz=200, vsr_blocks=260),            # 13
+        dict(n_out=70, n_in=520, d=8, k1=256, bits1=8, n_groups=3, col_scale=True, nnz=90),                  # 14
+        dict(n_out=40, n_in=512, d=8, k1=65536, bits1=16, cb_symmetry=1, col_scale=True, nnz=50, vsr_blocks=30),  # 15
+        dict(n_out=50, n_in=133, d=4, k1=64, bits1=6, k2=16, bits2=4, n_groups=2, cb_symmetry=1, n_ocols=7,
+             ko=32, bits_o=5, nnz=40, vsr_blocks=25),                                                         # 16
+        dict(n_out=45, n_in=300, d=12, k1=128, bits1=7, cb_symmetry=1, nnz=30, vsr_blocks=20),              # 17
+        dict(n_out=64, n_in=200, d=8, k1=4096, bits1=12, k2=256, bits2=8, n_groups=2, nnz=40, vsr_blocks=16,
+             n_ocols=9, ko=64, bits_o=6),                                                                     # 18
+        dict(n_out=33, n_in=96, d=8, k1=1024, bits1=10, n_groups=12, cb_symmetry=1, nnz=10),                 # 19 one position per group
     ]
     out = []
     for t, kw in enumerate(specs):
@@ -267,7 +277,7 @@ def run_gemm(vq, L, Xbits, xdt, ydt):
     return G.to_f64(Y)
 
 
-@pytest.mark.parametrize("t", [0, 1, 2, 4, 10, 11, 12])
+@pytest.mark.parametrize("t", [0, 1, 2, 4, 10, 11, 12, 13, 14, 15, 18, 19])
 @pytest.mark.parametrize("M", [1, 77, 256])
 def test_gemm_small(vq, t, M):
     L = SMALL[t]
@@ -277,6 +287,25 @@ def test_gemm_small(vq, t, M):
     Xb = synth.activations(rng, M, L.n_in, "bf16")
     Y = run_gemm(vq, L, Xb, "bf16", "f32")
     G.assert_close(Y, oracle.gemv_f64(L, synth.bits_to_f64(Xb, "bf16")), "f32", "gemm small")
+
+
+@pytest.mark.parametrize("M", [1, 300, 513, 1100])
+def test_gemm_fused_ragged_tiles(vq, M):
+    """The fused prefill (weight tiles dequantised in shared memory): 300 weight rows (three
+    128-row tiles, the last ragged), 200 columns (three whole K-blocks and a partial one), row and
+    column scales and CSR replacements; M covers one and two activation halves and several
+    512-row groups."""
+    import torch
+    rng = np.random.default_rng(4300 + M)
+    L = synth.random_layer(rng, 300, 200, 8, 256, 8, col_scale=True, cb_std=0.3, nnz=700, outlier_scale=1.0)
+    Xb = synth.activations(rng, M, L.n_in, "f16")
+    m = vq.VQLinear(L)
+    n0 = vq.vqlin_kernel_launches()
+    Y = m.gemm(G.torch_x(Xb, "f16"), out_dtype=torch.float32)
+    assert vq.vqlin_kernel_launches() - n0 == 1          # one fused kernel, no dequant pass
+    torch.cuda.synchronize()
+    assert vq.device_error() == 0
+    G.assert_close(G.to_f64(Y), oracle.gemv_f64(L, synth.bits_to_f64(Xb, "f16")), "f32", "fused gemm M=%d" % M)
 
 
 def test_gemm_prefill_sampled_rows(vq):
@@ -383,6 +412,12 @@ def cs_layers():
     L.codes = synth.pack_fields(fields, 16)
     L.fields = fields
     out.append(L)
+    # symmetric K = 65536 codebook (16384 stored entries) with VSR blocks, and 4 groups of a
+    # K = 4096 codebook (a 16384-entry virtual codebook): both take the codebook-stationary layout
+    out.append(synth.random_layer(rng, 600, 1024, 8, 65536, 16, cb_symmetry=1, col_scale=True, nnz=300,
+                                  vsr_blocks=500, name="cs_sym_vsr"))
+    out.append(synth.random_layer(rng, 2100, 768, 8, 4096, 12, n_groups=4, nnz=400, vsr_blocks=300,
+                                  name="cs_groups"))
     return out
 
 

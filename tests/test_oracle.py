@@ -175,6 +175,14 @@ CASES = [
     dict(n_out=3, n_in=30, d=6, k1=16, bits1=4, k2=5, bits2=3, n_ocols=7, ko=3, bits_o=2, nnz=4),
     dict(n_out=3, n_in=29, d=12, k1=32, bits1=5, col_scale=True, nnz=6),                    # d = 12, ragged tail
     dict(n_out=2, n_in=40, d=12, k1=256, bits1=8, k2=16, bits2=4, n_ocols=13, ko=7, bits_o=3, col_scale=True, nnz=5),
+    # codebook groups (VPTQ group_num), symmetric codebooks (SCVQ), VSR blocks (SCVQ)
+    dict(n_out=4, n_in=40, d=4, k1=16, bits1=4, n_groups=3, col_scale=True, nnz=4),         # 10 positions, 3 groups
+    dict(n_out=3, n_in=44, d=4, k1=8, bits1=3, k2=4, bits2=2, n_groups=4, n_ocols=4, ko=5, bits_o=3, nnz=3),
+    dict(n_out=5, n_in=24, d=8, k1=64, bits1=6, cb_symmetry=1, col_scale=True, nnz=6),
+    dict(n_out=4, n_in=30, d=6, k1=32, bits1=5, cb_symmetry=1, n_groups=2, k2=3, bits2=2, nnz=3),
+    dict(n_out=6, n_in=27, d=4, k1=16, bits1=4, col_scale=True, nnz=8, vsr_blocks=9),      # ragged tail block possible
+    dict(n_out=5, n_in=34, d=8, k1=64, bits1=6, cb_symmetry=1, n_groups=2, n_ocols=5, ko=6, bits_o=3, nnz=6,
+         vsr_blocks=6),
 ]
 
 
@@ -200,6 +208,110 @@ def test_dequant_matches_rational_brute_force(case):
         scale = sum(abs(float(Wq[i][j]) * x[b, j]) for i in range(L.n_out) for j in range(L.n_in))
         for i in range(L.n_out):
             assert abs(y[b, i] - float(yq[b][i])) <= 4 * L.n_in * 2.0**-53 * scale
+
+
+# ---------------------------------------------------------------- groups, symmetric codebooks, VSR
+def test_identical_group_codebooks_reduce_to_one_codebook():
+    """n_groups copies of the same codebook decode like the single codebook (VPTQ's group
+    partitioning with nothing to specialise)."""
+    rng = np.random.default_rng(120)
+    L1 = synth.random_layer(rng, 7, 80, 8, 32, 5, col_scale=True, nnz=9)
+    for G in (2, 3, 10):
+        LG = synth.LayerData(**{k: v for k, v in L1.__dict__.items()})
+        LG.n_groups = G
+        LG.codebook1 = np.tile(L1.codebook1, (G, 1))
+        assert (oracle.dequant_exact(LG) == oracle.dequant_exact(L1)).all()
+
+
+def test_group_boundaries_follow_the_position_ranges():
+    """Group g owns positions [g * ceil(n_sub / G), ...): with one-hot codebooks whose group g
+    entry is the value g + 1 everywhere, every decoded weight names its group."""
+    n_out, d, G, k1 = 3, 4, 3, 2
+    n_sub = 7                                         # groups of 3, 3, 1 positions
+    cb = np.concatenate([np.full((k1, d), g + 1.0) for g in range(G)])
+    L = synth.LayerData(n_out=n_out, n_in=n_sub * d, d=d, k1=k1, bits1=1,
+                        codes=synth.pack_fields(np.zeros((n_out, n_sub), np.uint32), 1),
+                        codebook1=synth.f16_bits(cb), n_groups=G)
+    W = oracle.dequant_f64(L)
+    want = np.repeat(np.array([1, 1, 1, 2, 2, 2, 3], float), d)
+    assert (W == want[None, :]).all()
+
+
+def test_symmetric_codebook_equals_its_expansion():
+    """A symmetric codebook decodes like the plain codebook of its k1 entries, built here with
+    numpy negation: pattern 0 +, 1 all -, 2 odd elements -, 3 even elements -."""
+    rng = np.random.default_rng(121)
+    for d, G in ((4, 1), (8, 2), (12, 1)):
+        L = synth.random_layer(rng, 6, 6 * d + 3, d, 16, 4, cb_symmetry=1, n_groups=G, col_scale=True, nnz=5)
+        base = L.codebook1.view(np.float16).astype(np.float64).reshape(G, 4, d)
+        sign = np.ones((4, d))
+        sign[1] = -1
+        sign[2, 1::2] = -1
+        sign[3, 0::2] = -1
+        full = (sign[None, :, None, :] * base[:, None, :, :]).reshape(G * 16, d)
+        P = synth.LayerData(**{k: v for k, v in L.__dict__.items()})
+        P.cb_symmetry = 0
+        P.codebook1 = synth.f16_bits(full)
+        assert (oracle.dequant_exact(L) == oracle.dequant_exact(P)).all()
+
+
+def _vsr_as_csr(L):
+    """The same layer with every VSR block written as d CSR entries (main columns, REPLACE)."""
+    main = np.array([j for j in range(L.n_in) if j not in set(L.ocols.tolist())])
+    rows, cols, vals = [], [], []
+    for i in range(L.n_out):
+        if L.nnz:
+            for e in range(L.row_ptr[i], L.row_ptr[i + 1]):
+                rows.append(i); cols.append(int(L.col_idx[e])); vals.append(int(L.values[e]))
+        for b in range(L.vsr_row_ptr[i], L.vsr_row_ptr[i + 1]):
+            for t in range(L.d):
+                q = int(L.vsr_pos[b]) * L.d + t
+                if q < main.size:
+                    rows.append(i); cols.append(int(main[q])); vals.append(int(L.vsr_values[b, t]))
+    rp, ci, v = synth.csr_from_positions(L.n_out, np.array(rows), np.array(cols), np.array(vals, np.uint16))
+    C = synth.LayerData(**{k: v for k, v in L.__dict__.items()})
+    C.row_ptr, C.col_idx, C.values = rp, ci, v
+    C.vsr_row_ptr = C.vsr_pos = C.vsr_values = None
+    return C
+
+
+def test_vsr_blocks_equal_their_csr_entries():
+    rng = np.random.default_rng(122)
+    for kw in (dict(d=8, n_ocols=0), dict(d=4, n_ocols=5), dict(d=12, n_ocols=3)):
+        L = synth.random_layer(rng, 9, 101, kw["d"], 64, 6, n_ocols=kw["n_ocols"], ko=8, bits_o=3,
+                               col_scale=True, nnz=25, vsr_blocks=14)
+        assert L.vsr_nblocks == 14
+        C = _vsr_as_csr(L)
+        assert (oracle.dequant_exact(L) == oracle.dequant_exact(C)).all()
+        x = rng.standard_normal((2, L.n_in))
+        assert np.array_equal(oracle.gemv_f64(L, x), oracle.gemv_f64(C, x))
+
+
+def test_vsr_full_rows_are_dense_rows():
+    rng = np.random.default_rng(123)
+    d, n_in = 8, 40
+    L = synth.random_layer(rng, 3, n_in, d, 16, 4, col_scale=True, nnz=0)
+    V = rng.normal(0, 1, (3, n_in)).astype(np.float16)
+    L.vsr_row_ptr = (np.arange(4) * (n_in // d)).astype(np.int32)
+    L.vsr_pos = np.tile(np.arange(n_in // d), 3).astype(np.int32)
+    L.vsr_values = V.reshape(-1, d).view(np.uint16)
+    assert (oracle.dequant_exact(L) == V.view(np.uint16)).all()
+
+
+def test_malformed_vsr_is_reported():
+    rng = np.random.default_rng(124)
+    L = synth.random_layer(rng, 4, 32, 8, 16, 4, nnz=0, vsr_blocks=3)
+    bad = synth.LayerData(**{k: v for k, v in L.__dict__.items()})
+    bad.vsr_pos = L.vsr_pos.copy(); bad.vsr_pos[0] = 4                      # position >= n_sub
+    with pytest.raises(oracle.OracleError):
+        oracle.dequant_exact(bad)
+    row = int(np.nonzero(np.diff(L.vsr_row_ptr))[0][0])
+    s0 = int(L.vsr_pos[L.vsr_row_ptr[row]])
+    over = synth.LayerData(**{k: v for k, v in L.__dict__.items()})
+    over.row_ptr = np.zeros(5, np.int32); over.row_ptr[row + 1:] = 1
+    over.col_idx = np.array([s0 * 8 + 3], np.int32); over.values = synth.f16_bits([1.0])   # inside a block
+    with pytest.raises(oracle.OracleError):
+        oracle.dequant_exact(over)
 
 
 def test_rows_subset_matches_full():
