@@ -401,20 +401,29 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
     }
   }
 
-  // tensor-core decode layout (see vqlin_internal.cuh).  With codebook groups its fields hold
-  // g * k1 + i1 | (g * k2 + i2) << tc_b1, widened to the next width its kernels take.
+  // tensor-core decode layout (see vqlin_internal.cuh).  Its kernels work on 8-wide parts: for
+  // d != 8 every sub-vector becomes V = ceil(d / 8) parts, zero-padded, each with its own entry of
+  // a padded codebook (entry k, part h at k * V + h); x' is then staged through a map from the
+  // layout's columns to the layer's (padding to none).  With codebook groups (or parts) the fields
+  // hold (g * k1 + i1) * V + h | ((g * k2 + i2) * V + h) << tc_b1, widened to the next width the
+  // kernels take.  Outlier-column blocks are decoded there only at d = 8.
   std::vector<uint8_t> tcodes;
+  std::vector<uint16_t> tcb1, tcb2;                 // padded codebooks (d != 8 only)
+  std::vector<int32_t> tcmap;                       // layout column -> layer column or -1 (d != 8)
   int32_t n_ls = 0;
   int64_t tstride = 0;
+  const int V = (d + 7) / 8;
+  const int32_t tc_nsub = n_sub * V;
   int tc_b1 = D->bits1, tc_w = w;
-  if (G > 1) {
+  if (G > 1 || V > 1) {
     auto bits_for = [](int64_t n) { int b = 1; while ((1ll << b) < n) ++b; return b; };
-    tc_b1 = bits_for((int64_t)G * D->k1);
-    const int need = tc_b1 + (D->k2 ? bits_for((int64_t)G * D->k2) : 0);
+    tc_b1 = bits_for((int64_t)G * D->k1 * V);
+    const int need = tc_b1 + (D->k2 ? bits_for((int64_t)G * D->k2 * V) : 0);
     tc_w = need <= 8 ? 8 : need <= 12 ? 12 : need <= 16 ? 16 : need <= 24 ? 24 : need <= 32 ? 32 : 0;
   }
-  if (d == 8 && n_sub > 0 && (tc_w == 8 || tc_w == 12 || tc_w == 16 || tc_w == 24 || tc_w == 32)) {
-    n_ls = (int32_t)ceil_div(n_sub, 64);
+  const bool tc_geom = d == 8 || D->n_ocols == 0;
+  if (tc_geom && n_sub > 0 && (tc_w == 8 || tc_w == 12 || tc_w == 16 || tc_w == 24 || tc_w == 32)) {
+    n_ls = (int32_t)ceil_div(tc_nsub, 64);
     tstride = (int64_t)n_ls * 8 * tc_w;
     const int64_t rows_pad = round_up(D->n_out, 16);
     tcodes.assign((size_t)(rows_pad * tstride), 0);
@@ -424,15 +433,33 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
       for (int32_t ls = 0; ls < n_ls; ++ls)
         for (int t = 0; t < 4; ++t)
           for (int ps = 0; ps < 16; ++ps) {
-            int32_t sv = 64 * ls + 4 * ps + t;
-            if (sv >= n_sub) continue;   // padding fields stay 0 (a valid index; x' is 0 there)
+            const int32_t vsv = 64 * ls + 4 * ps + t;          // part index in the layout
+            if (vsv >= tc_nsub) continue;   // padding fields stay 0 (a valid index; x' is 0 there)
+            const int32_t sv = vsv / V, h = vsv - sv * V;
             uint32_t f = host_field(row, sv, w);
-            if (G > 1) {
+            if (G > 1 || V > 1) {
               const uint32_t g = (uint32_t)(sv / g_size);
-              f = (g * (uint32_t)D->k1 + (f & m1)) | ((D->k2 ? g * (uint32_t)D->k2 + (f >> D->bits1) : 0u) << tc_b1);
+              f = ((g * (uint32_t)D->k1 + (f & m1)) * (uint32_t)V + (uint32_t)h) |
+                  ((D->k2 ? (g * (uint32_t)D->k2 + (f >> D->bits1)) * (uint32_t)V + (uint32_t)h : 0u) << tc_b1);
             }
             host_put_field(dst, (int64_t)ls * 64 + t * 16 + ps, tc_w, f);
           }
+    }
+    if (d != 8) {
+      auto pad = [&](const std::vector<uint8_t>& cb, int64_t entries, std::vector<uint16_t>& out) {
+        const uint16_t* c = as<uint16_t>(cb);
+        out.assign((size_t)entries * V * 8, 0);
+        for (int64_t k = 0; k < entries; ++k)
+          for (int h = 0; h < V; ++h)
+            for (int e = 0; e < 8 && 8 * h + e < d; ++e) out[((size_t)k * V + h) * 8 + e] = c[(size_t)k * d + 8 * h + e];
+      };
+      pad(cb1, (int64_t)G * D->k1, tcb1);
+      if (D->k2) pad(cb2, (int64_t)G * D->k2, tcb2);
+      tcmap.assign((size_t)tc_nsub * 8, -1);
+      for (int32_t c = 0; c < tc_nsub * 8; ++c) {
+        const int32_t vsv = c / 8, k = c % 8, sv = vsv / V, h = vsv - sv * V, e = 8 * h + k, q = sv * d + e;
+        if (e < d && q < n_main) tcmap[c] = q;      // no outlier block here, so main column q is column q
+      }
     }
   }
 
@@ -614,6 +641,12 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
   L.tstride = tstride;
   L.tc_w = tcodes.empty() ? 0 : tc_w;
   L.tc_bits1 = tc_b1;
+  L.tc_nsub = tcodes.empty() ? 0 : tc_nsub;
+  L.tc_k1 = G * D->k1 * V;
+  L.tc_k2 = G * D->k2 * V;
+  L.tc_cb1 = tcb1.empty() ? L.cb1 : up.put<__half>(tcb1.data(), tcb1.size() * 2);
+  L.tc_cb2 = tcb2.empty() ? L.cb2 : up.put<__half>(tcb2.data(), tcb2.size() * 2);
+  L.tc_colmap = tcmap.empty() ? nullptr : up.put<int32_t>(tcmap.data(), tcmap.size() * 4);
   L.tcodes_rows = tcodes.empty() ? 0 : (int32_t)round_up(D->n_out, 16);
   if (up.st == VQLIN_OK) up.st = cuda_status(cudaStreamSynchronize((cudaStream_t)stream), "create sync");
   if (up.st != VQLIN_OK) {

@@ -119,8 +119,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
   // ---- shared memory carve-up
   unsigned char* sp = smem;
   uint4* cb1s = reinterpret_cast<uint4*>(sp);
-  uint4* cb2s = cb1s + (CB_SMEM ? (size_t)L.n_groups * L.k1 * COPIES : 0);
-  sp = reinterpret_cast<unsigned char*>(cb2s + (CB_SMEM ? (size_t)L.n_groups * L.k2 * COPIES : 0));
+  uint4* cb2s = cb1s + (CB_SMEM ? (size_t)L.tc_k1 * COPIES : 0);
+  sp = reinterpret_cast<unsigned char*>(cb2s + (CB_SMEM ? (size_t)L.tc_k2 * COPIES : 0));
   __half* xh = reinterpret_cast<__half*>(sp);                      // [batch][xs_cols]
   __half* xl = xh + (size_t)a.batch * a.xs_cols;
   float* red = reinterpret_cast<float*>(xl + (size_t)a.batch * a.xs_cols);   // [rtt][16][8*NT]
@@ -133,11 +133,11 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
 
   // ---- codebooks into shared memory (COPIES interleaved copies: entry k of copy c at k*COPIES + c)
   if (CB_SMEM) {
-    const uint4* c1 = reinterpret_cast<const uint4*>(L.cb1);
-    for (int i = threadIdx.x; i < L.n_groups * L.k1 * COPIES; i += THREADS) cb1s[i] = __ldg(c1 + i / COPIES);
+    const uint4* c1 = reinterpret_cast<const uint4*>(L.tc_cb1);
+    for (int i = threadIdx.x; i < L.tc_k1 * COPIES; i += THREADS) cb1s[i] = __ldg(c1 + i / COPIES);
     if (L.k2) {
-      const uint4* c2 = reinterpret_cast<const uint4*>(L.cb2);
-      for (int i = threadIdx.x; i < L.n_groups * L.k2 * COPIES; i += THREADS) cb2s[i] = __ldg(c2 + i / COPIES);
+      const uint4* c2 = reinterpret_cast<const uint4*>(L.tc_cb2);
+      for (int i = threadIdx.x; i < L.tc_k2 * COPIES; i += THREADS) cb2s[i] = __ldg(c2 + i / COPIES);
     }
   }
   // ---- layer-only prefetch for this block's first task, before the wait: the index words of
@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
       const int b = i / groups, q = (i - b * groups) * 8;
       const int qq = col0 + q;
       float v[8];
-      if (!L.colmap && a.xt != VQLIN_F32 && qq + 8 <= L.n_main && (L.n_in & 7) == 0) {
+      if (!L.colmap && !L.tc_colmap && a.xt != VQLIN_F32 && qq + 8 <= L.n_main && (L.n_in & 7) == 0) {
         uint4 u = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const unsigned short*>(a.x) +
                                                         (int64_t)b * L.n_in + qq));
         const unsigned short* hs = reinterpret_cast<const unsigned short*>(&u);
@@ -222,7 +222,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const int c = qq + k;
-          jj[k] = c < L.n_main ? (L.colmap ? L.colmap[c] : c) : -1;
+          jj[k] = L.tc_colmap ? (c < L.tc_nsub * 8 ? L.tc_colmap[c] : -1) : (c < L.n_main ? (L.colmap ? L.colmap[c] : c) : -1);
         }
 #pragma unroll
         for (int k = 0; k < 8; ++k) v[k] = jj[k] >= 0 ? load_as_float(a.x, a.xt, (int64_t)b * L.n_in + jj[k]) : 0.f;
@@ -343,16 +343,16 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemv_tc(Args a) {
             c0[j] = cb1s[(f0 & m1) * COPIES + (lane & (COPIES - 1))];
             c1[j] = cb1s[(f1 & m1) * COPIES + (lane & (COPIES - 1))];
           } else {
-            c0[j] = __ldg(reinterpret_cast<const uint4*>(L.cb1) + (f0 & m1));
-            c1[j] = __ldg(reinterpret_cast<const uint4*>(L.cb1) + (f1 & m1));
+            c0[j] = __ldg(reinterpret_cast<const uint4*>(L.tc_cb1) + (f0 & m1));
+            c1[j] = __ldg(reinterpret_cast<const uint4*>(L.tc_cb1) + (f1 & m1));
           }
           if (L.k2) {
             if (CB_SMEM) {
               e0[j] = cb2s[(f0 >> L.tc_bits1) * COPIES + (lane & (COPIES - 1))];
               e1[j] = cb2s[(f1 >> L.tc_bits1) * COPIES + (lane & (COPIES - 1))];
             } else {
-              e0[j] = __ldg(reinterpret_cast<const uint4*>(L.cb2) + (f0 >> L.tc_bits1));
-              e1[j] = __ldg(reinterpret_cast<const uint4*>(L.cb2) + (f1 >> L.tc_bits1));
+              e0[j] = __ldg(reinterpret_cast<const uint4*>(L.tc_cb2) + (f0 >> L.tc_bits1));
+              e1[j] = __ldg(reinterpret_cast<const uint4*>(L.tc_cb2) + (f1 >> L.tc_bits1));
             }
           }
         }
@@ -442,8 +442,8 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) k_gemv_wt(Args a) {
   const Layer& L = a.L;
   extern __shared__ __align__(16) unsigned char smem[];
   uint4* cb1s = reinterpret_cast<uint4*>(smem);
-  uint4* cb2s = cb1s + (CB_SMEM ? (size_t)L.n_groups * L.k1 * COPIES : 0);
-  __half* xh = reinterpret_cast<__half*>(cb2s + (CB_SMEM ? (size_t)L.n_groups * L.k2 * COPIES : 0));   // [batch][xs_cols]
+  uint4* cb2s = cb1s + (CB_SMEM ? (size_t)L.tc_k1 * COPIES : 0);
+  __half* xh = reinterpret_cast<__half*>(cb2s + (CB_SMEM ? (size_t)L.tc_k2 * COPIES : 0));   // [batch][xs_cols]
   __half* xl = xh + (size_t)a.batch * a.xs_cols;
   float* xo = reinterpret_cast<float*>(xl + (size_t)a.batch * a.xs_cols);               // [BP][n_sub_o*8]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -452,11 +452,11 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) k_gemv_wt(Args a) {
   const uint32_t m1 = (1u << L.tc_bits1) - 1u;   // first-stage bits of the tensor-core layout
 
   if (CB_SMEM) {
-    const uint4* c1 = reinterpret_cast<const uint4*>(L.cb1);
-    for (int i = threadIdx.x; i < L.n_groups * L.k1 * COPIES; i += WT_THREADS) cb1s[i] = __ldg(c1 + i / COPIES);
+    const uint4* c1 = reinterpret_cast<const uint4*>(L.tc_cb1);
+    for (int i = threadIdx.x; i < L.tc_k1 * COPIES; i += WT_THREADS) cb1s[i] = __ldg(c1 + i / COPIES);
     if (L.k2) {
-      const uint4* c2 = reinterpret_cast<const uint4*>(L.cb2);
-      for (int i = threadIdx.x; i < L.n_groups * L.k2 * COPIES; i += WT_THREADS) cb2s[i] = __ldg(c2 + i / COPIES);
+      const uint4* c2 = reinterpret_cast<const uint4*>(L.tc_cb2);
+      for (int i = threadIdx.x; i < L.tc_k2 * COPIES; i += WT_THREADS) cb2s[i] = __ldg(c2 + i / COPIES);
     }
   }
   // x (and the accumulator) belong to the previous grid until it completes
@@ -484,7 +484,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) k_gemv_wt(Args a) {
       const int b = i / groups, q = (i - b * groups) * 8;
       const int qq = col0 + q;                         // main-column index of this group
       float v[8];
-      if (!L.colmap && a.xt != VQLIN_F32 && qq + 8 <= L.n_main && (L.n_in & 7) == 0) {
+      if (!L.colmap && !L.tc_colmap && a.xt != VQLIN_F32 && qq + 8 <= L.n_main && (L.n_in & 7) == 0) {
         uint4 u = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const unsigned short*>(a.x) +
                                                         (int64_t)b * L.n_in + qq));
         const unsigned short* hs = reinterpret_cast<const unsigned short*>(&u);
@@ -500,7 +500,9 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) k_gemv_wt(Args a) {
       } else {
         int jj[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) jj[k] = qq + k < L.n_main ? (L.colmap ? L.colmap[qq + k] : qq + k) : -1;
+        for (int k = 0; k < 8; ++k)
+          jj[k] = L.tc_colmap ? (qq + k < L.tc_nsub * 8 ? L.tc_colmap[qq + k] : -1)
+                              : (qq + k < L.n_main ? (L.colmap ? L.colmap[qq + k] : qq + k) : -1);
 #pragma unroll
         for (int k = 0; k < 8; ++k) v[k] = jj[k] >= 0 ? load_as_float(a.x, a.xt, (int64_t)b * L.n_in + jj[k]) : 0.f;
         if (L.cs) {
@@ -527,14 +529,15 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) k_gemv_wt(Args a) {
   const int n_side = has_side ? (L.n_out + 7) / 8 : 0;      // sparse / outlier tasks of 8 rows
   const int gpc = (ks_end - ks_beg + a.wt_spt - 1) / a.wt_spt;   // slab groups of this chunk
   const int n_mt = n_rt * gpc;                                    // this chunk's MMA tasks
-  // the sparse / outlier tasks first (spread over every block), then this chunk's MMA tasks
-  // (spread over the chunk's blocks)
-  const int side_beg = blockIdx.x * NW + warp, side_step = gridDim.x * NW;
-  const int n_side_mine = side_beg < n_side ? (n_side - side_beg + side_step - 1) / side_step : 0;
-  const int total = n_side_mine + (jb * NW + warp < n_mt ? (n_mt - jb * NW - warp + a.wt_bpc * NW - 1) / (a.wt_bpc * NW) : 0);
-  for (int it = 0; it < total; ++it) {
-    const int task = it < n_side_mine ? side_beg + it * side_step : -1;
-    if (task >= 0) {
+  // One task space per chunk, dealt round-robin over the chunk's warps: first the chunk's share of
+  // the sparse / outlier tasks (side task ch, ch + nch, ...), then its MMA tasks, so every warp
+  // gets the same number of tasks whichever kind they are.
+  const int nch = a.wt_nch;
+  const int n_side_c = n_side / nch + (ch < n_side % nch ? 1 : 0);
+  const int total_c = n_side_c + n_mt;
+  for (int tk = jb * NW + warp; tk < total_c; tk += a.wt_bpc * NW) {
+    if (tk < n_side_c) {
+      const int task = ch + tk * nch;                   // side task: rows 8 task .. +7
       // ---- fused sparse correction and outlier block for rows 8*task .. +8 (4 lanes per row)
       const int64_t row = (int64_t)task * 8 + (lane >> 2);
       const int sub = lane & 3;
@@ -573,9 +576,10 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) k_gemv_wt(Args a) {
       continue;
     }
     // ---- MMA task: row tile rt over the kernel slabs of slab group sg of this chunk
-    const int mt = jb * NW + warp + (it - n_side_mine) * a.wt_bpc * NW;
+    const int mt = tk - n_side_c;
     const int rt = mt / gpc, sg = mt - rt * gpc;
-    const int kb0 = ks_beg + sg * a.wt_spt, kb1 = min(kb0 + a.wt_spt, ks_end);
+    // one slab per task at batch <= 8 (NT <= 2), known at compile time; several at batch > 8
+    const int kb0 = ks_beg + sg * a.wt_spt, kb1 = NT <= 2 ? kb0 + 1 : min(kb0 + a.wt_spt, ks_end);
     const int64_t R0 = (int64_t)rt * 16 + g;
     constexpr int NWORDS = (2 * W / NT + 3) / 4 + 1;
     const float r0 = (L.rs && R0 < L.n_out) ? __half2float(L.rs[R0]) : 1.f;
@@ -608,16 +612,16 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) k_gemv_wt(Args a) {
           c0[j] = cb1s[(f0 & m1) * COPIES + (lane & (COPIES - 1))];
           c1[j] = cb1s[(f1 & m1) * COPIES + (lane & (COPIES - 1))];
         } else {
-          c0[j] = __ldg(reinterpret_cast<const uint4*>(L.cb1) + (f0 & m1));
-          c1[j] = __ldg(reinterpret_cast<const uint4*>(L.cb1) + (f1 & m1));
+          c0[j] = __ldg(reinterpret_cast<const uint4*>(L.tc_cb1) + (f0 & m1));
+          c1[j] = __ldg(reinterpret_cast<const uint4*>(L.tc_cb1) + (f1 & m1));
         }
         if (L.k2) {
           if (CB_SMEM) {
             e0[j] = cb2s[(f0 >> L.tc_bits1) * COPIES + (lane & (COPIES - 1))];
             e1[j] = cb2s[(f1 >> L.tc_bits1) * COPIES + (lane & (COPIES - 1))];
           } else {
-            e0[j] = __ldg(reinterpret_cast<const uint4*>(L.cb2) + (f0 >> L.tc_bits1));
-            e1[j] = __ldg(reinterpret_cast<const uint4*>(L.cb2) + (f1 >> L.tc_bits1));
+            e0[j] = __ldg(reinterpret_cast<const uint4*>(L.tc_cb2) + (f0 >> L.tc_bits1));
+            e1[j] = __ldg(reinterpret_cast<const uint4*>(L.tc_cb2) + (f1 >> L.tc_bits1));
           }
         }
       }
@@ -756,8 +760,7 @@ static size_t gemv_acc_bytes(const Layer& L, int batch) {
 }
 
 bool tc_supported(const Layer& L) {
-  return L.d == 8 && L.tcodes != nullptr &&
-         (L.tc_w == 8 || L.tc_w == 12 || L.tc_w == 16 || L.tc_w == 24 || L.tc_w == 32);
+  return L.tcodes != nullptr && (L.tc_w == 8 || L.tc_w == 12 || L.tc_w == 16 || L.tc_w == 24 || L.tc_w == 32);
 }
 
 size_t gemv_workspace_bytes(const Layer& L, int batch) {
@@ -791,11 +794,11 @@ cudaError_t launch_gemv_tc(const Layer& L, const void* x, vqlin_dtype xt, int ba
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const size_t smem_max = 227 * 1024;
   // codebooks: as many interleaved copies (<= 8) as fit next to x'
-  const size_t cb_entries = (size_t)L.n_groups * ((size_t)L.k1 + L.k2);
+  const size_t cb_entries = (size_t)L.tc_k1 + L.tc_k2;
   Args a;
   a.L = L; a.x = x; a.xt = xt; a.batch = batch; a.y = y; a.yt = yt; a.acc = nullptr;
   a.wt_cs = 0; a.wt_nch = 1; a.wt_bpc = 1; a.wt_spt = 1;   // set by the warp-task plan below
-  a.n_kslabs = (L.n_sub + KSV - 1) / KSV;
+  a.n_kslabs = (L.tc_nsub + KSV - 1) / KSV;
   a.ks = a.n_kslabs < WARPS ? a.n_kslabs : WARPS;
   // round ks down to a divisor of WARPS so that rtt * ks == WARPS when several row tiles share a CTA
   while (WARPS % a.ks) --a.ks;
@@ -884,7 +887,7 @@ cudaError_t launch_gemv_tc(const Layer& L, const void* x, vqlin_dtype xt, int ba
         const int64_t slab_tasks = (int64_t)n_rt * a.n_kslabs, target = 3ll * grid * nw;
         spt = (int)((slab_tasks + target - 1) / target);
         if (spt > cs) spt = cs;
-        if (spt < 1) spt = 1;
+        if (spt < 1 || NT <= 2) spt = 1;               // the NT <= 2 kernels take one slab per task
       }
       w.wt_cs = cs; w.wt_nch = nch; w.wt_bpc = bpc; w.wt_spt = spt;
       // plan checks: every chunk's slabs are staged, and the grid is whole chunks of blocks

@@ -53,8 +53,15 @@ struct Layer {
   // With codebook groups the fields of this layout hold g * k1 + i1 (and g * k2 + i2 above
   // tc_bits1), widened to tc_w bits, so these kernels index the concatenated codebooks directly;
   // with one group tc_w = w and tc_bits1 = bits1.
+  // For d != 8 (no outlier block) the layout works on 8-wide parts: tc_nsub = n_sub * ceil(d/8)
+  // parts per row, decoded with the zero-padded codebooks tc_cb1 / tc_cb2 (tc_k1 / tc_k2 entries,
+  // entry k part h at k * ceil(d/8) + h), and x' staged through tc_colmap (layout column -> layer
+  // column or -1).  At d = 8: tc_nsub = n_sub, tc_cb = cb, tc_colmap = null.
   const uint8_t* tcodes;
-  int32_t tc_w, tc_bits1;
+  int32_t tc_w, tc_bits1, tc_nsub, tc_k1, tc_k2;
+  const __half* tc_cb1;
+  const __half* tc_cb2;
+  const int32_t* tc_colmap;
   int32_t n_ls;                         // layout slabs per row
   int32_t tcodes_rows;                  // rows allocated in tcodes (n_out rounded up to 16)
   int64_t tstride;                      // bytes per row = n_ls * 8 * tc_w
