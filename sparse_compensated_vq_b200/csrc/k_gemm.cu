@@ -269,43 +269,57 @@ __global__ void __launch_bounds__(THREADS, 1)
 //
 // Orientation.  The MMA's M side is the weight: a CTA owns 128 weight rows (outputs) and 512
 // activation rows, Y^T[128][512] = W_tile[128][K] * X_tile[512][K]^T, as two N = 256
-// accumulators that fill the 512 TMEM columns.  Each weight row is then gathered once per 512
-// activation rows (the TMEM limit), not once per activation tile of a conventional tiling.
+// accumulators that fill the 512 TMEM columns.
 //
-// Warp roles (10 warps):
+// Sharing the weight tile.  The CS CTAs of a thread-block cluster (CS = 2 up to 1024 activation
+// rows, 4 beyond) own the same 128 weight rows and different 512-row activation groups (a CTA past
+// the last activation row still converts and shares its part).  Each gathers and
+// converts only its 128 / CS rows of every weight K-block into its own slot, and one thread copies
+// them into the same slot of each peer (cp.async.bulk shared::cta -> shared::cluster, completing
+// on the peer's slot barrier).  So every weight element is gathered
+// and converted once per 512 * CS activation rows.  A slot is rewritten only when every CTA's MMA
+// has finished with it: the MMA returns a slot with one tcgen05.commit multicast to the slot's
+// "cluster empty" barrier in every CTA of the cluster.
+//
+// Warp roles (11 warps):
 //   warp 0      TMA producer of the activation tiles: 256 rows x 64 k (one 128-byte swizzle row
 //               per activation row) into a 5-slot ring of half K-blocks;
 //   warp 1      allocates the 512 TMEM columns; one lane issues tcgen05.mma.kind::f16 (M = 128,
 //               N = 256, K = 16), four per half K-block, and returns ring slots with
 //               tcgen05.commit;
-//   warps 2-9   weight producers, then the epilogue.  Thread p owns weight row p % 128 and the
-//               sub-vectors 4 (p / 128) .. +3 of every K-block (64 columns = 8 sub-vectors).
-//               For K-block kb it reads its four index fields, copies the four centroids with
-//               cp.async straight to their 128-byte-swizzled places in the weight slot (chunk
-//               s ^ (row % 8) of the row's 128 bytes, the layout a TMA 128B-swizzle load makes),
-//               and, once they have landed, converts them in place to the exact fp16 weight
+//   warp 2      one lane copies this CTA's rows of each weight K-block to the peers once its
+//               producers have written them, and arms the slot's full barrier for the peers' bytes;
+//   warps 3-10  weight producers, then the epilogue.  A producer warp owns 16 / CS consecutive
+//               rows of this CTA's part (128 / CS rows); 2 CS lanes share a row, each with 4 / CS
+//               of the row's 8 sub-vectors in a K-block (64 columns).  Three K-blocks ahead a lane
+//               gathers its centroids into registers (index fields loaded two steps earlier
+//               still).  For K-block kb it converts them to the exact fp16 weight
 //               fp16(r_i c_j C[k][t]) (C r_i is exact in fp32; the product with c_j is rounded to
 //               odd in fp32, so the final fp16 rounding is the correctly rounded one, as in the
-//               exact dequantisation), writes the CSR values of its columns over them (REPLACE),
-//               makes the writes visible to the tensor core (fence.proxy.async) and arrives on
-//               the slot's barrier.  The weight tile is therefore bit for bit the dequantised W.
+//               exact dequantisation) and puts the VSR blocks of its sub-vectors in their places
+//               (REPLACE), all while the slot may still be in use.  Once the slot is free it stores
+//               them to their 128-byte-swizzled places (chunk s ^ (row % 8) of the row's 128
+//               bytes, the layout a TMA 128B-swizzle load makes), writes the CSR values of its
+//               columns over them (REPLACE) and makes the writes visible to the async proxy
+//               (fence.proxy.async).  The weight tile is therefore bit for bit the dequantised W.
 // Every mbarrier wait is bounded (1 s); on expiry the kernel records an error code, stops,
-// waits (bounded) for its own copies, frees TMEM and returns.
+// waits (bounded) for its own copies, frees TMEM and returns.  Every thread reaches the cluster
+// barriers at start and end.
 constexpr int FA_STAGES = 4, FB_STAGES = 5;
 constexpr int FA_BYTES = 128 * 64 * 2;             // 16 KB weight slot
 constexpr int FB_BYTES = 256 * 64 * 2;             // 32 KB activation half-slot
 constexpr int F_PROD_WARPS = 8;
-constexpr int F_THREADS = (2 + F_PROD_WARPS) * 32;
-constexpr int F_LOOKAHEAD = FA_STAGES - 1;         // K-blocks of gathers in flight per thread
+constexpr int F_THREADS = (3 + F_PROD_WARPS) * 32;
 constexpr int F_ROWS = 128, F_XROWS = 512;
 constexpr size_t F_SMEM_BYTES = 1024 + (size_t)FA_STAGES * FA_BYTES + (size_t)FB_STAGES * FB_BYTES + 256;
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+// 16-byte global load that is not kept in L1 (a centroid gather: no reuse worth caching)
+__device__ __forceinline__ uint4 ldg_nc_na(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // fp32 product rounded to odd: toward zero, last bit forced to 1 when inexact (the exact error
 // comes from a fused multiply-add).  Rounding that to fp16 gives the correctly rounded product.
@@ -316,68 +330,89 @@ __device__ __forceinline__ float rto_mul_f32(float a, float b) {
   return p;
 }
 
-// The four index fields of sub-vectors kb*8 + 4*hs .. +3 of one packed row: they occupy the w/2
-// bytes at byte kb*w + hs*w/2 (eight fields of a K-block are w bytes).  One vector load for
-// W = 8, 16, 32; three 32-bit loads of the K-block's w bytes for W = 12, 24; field by field
-// otherwise (W = 0: any width).
-template <int W>
-__device__ __forceinline__ void load_fields4(const uint8_t* row, int kb, int hs, int w, uint32_t* f) {
-  if constexpr (W == 8) {
-    const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(row + kb * 8 + hs * 4));
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// this CTA's shared address as seen in cluster CTA `rank`
+__device__ __forceinline__ uint32_t peer_addr(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+
+// The SPT index fields of sub-vectors kb*8 + SPT*j .. +SPT-1 of one packed row: SPT*w/8 bytes at
+// byte kb*w + j*SPT*w/8 (the eight fields of a K-block are w bytes).  One load when w is 8, 16 or
+// 32 (the row stride, a multiple of 16 bytes, and the 16 bytes of padding after the array cover
+// the K-block past the last sub-vector); field by field otherwise (W = 0: any width), fields at
+// or past n_sub reading as 0.
+template <int W, int SPT>
+__device__ __forceinline__ void load_fields(const uint8_t* row, int kb, int j, int w, int n_sub, uint32_t* f) {
+  constexpr int BYTES = SPT * W / 8;
+  const uint8_t* p = row + kb * W + j * BYTES;
+  if constexpr (W == 8 || W == 16 || W == 32) {
+    uint32_t v[SPT * W / 32 > 0 ? SPT * W / 32 : 1];
+    if constexpr (BYTES == 1) v[0] = __ldg(p);
+    else if constexpr (BYTES == 2) v[0] = __ldg(reinterpret_cast<const unsigned short*>(p));
+    else if constexpr (BYTES == 4) v[0] = __ldg(reinterpret_cast<const uint32_t*>(p));
+    else if constexpr (BYTES == 8) { const uint2 t = __ldg(reinterpret_cast<const uint2*>(p)); v[0] = t.x; v[1] = t.y; }
+    else { const uint4 t = __ldg(reinterpret_cast<const uint4*>(p)); v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w; }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) f[u] = (v >> (8 * u)) & 0xFFu;
-  } else if constexpr (W == 16) {
-    const uint2 v = __ldg(reinterpret_cast<const uint2*>(row + kb * 16 + hs * 8));
-    f[0] = v.x & 0xFFFFu; f[1] = v.x >> 16; f[2] = v.y & 0xFFFFu; f[3] = v.y >> 16;
-  } else if constexpr (W == 32) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(row + kb * 32 + hs * 16));
-    f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
-  } else if constexpr (W == 12 || W == 24) {
-    // W = 12: the K-block's 12 bytes (fields at bits 12 (4 hs + u)); W = 24: this half's 12 bytes
-    // (fields at bits 24 u); either way three 4-byte-aligned words
-    const uint32_t* p = reinterpret_cast<const uint32_t*>(row + kb * W + (W == 24 ? hs * 12 : 0));
-    const uint32_t a = __ldg(p), b = __ldg(p + 1), c = __ldg(p + 2);
-    const unsigned long long lo = (unsigned long long)a | ((unsigned long long)b << 32);
-    const unsigned long long hi = (unsigned long long)b | ((unsigned long long)c << 32);
-    constexpr uint32_t mask = (1u << W) - 1u;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int bit = (W == 12 ? 4 * hs + u : u) * W;
-      f[u] = (uint32_t)((bit <= 64 - W ? (lo >> bit) : (hi >> (bit - 32))) & mask);
+    for (int u = 0; u < SPT; ++u) {
+      const int bit = u * W;
+      f[u] = W == 32 ? v[u] : (v[bit >> 5] >> (bit & 31)) & ((1u << (W & 31)) - 1u);
     }
   } else {
 #pragma unroll
-    for (int u = 0; u < 4; ++u) f[u] = read_field(row, (int64_t)kb * 8 + 4 * hs + u, w);
+    for (int u = 0; u < SPT; ++u) {
+      const int sv = kb * 8 + SPT * j + u;
+      f[u] = sv < n_sub ? read_field(row, sv, w) : 0u;
+    }
   }
 }
 
-template <int W>
+template <int W, int CS>
 __global__ void __launch_bounds__(F_THREADS, 1)
     k_gemm_vq(const __grid_constant__ CUtensorMap map_x, const Layer L, int64_t M, void* __restrict__ Y,
               vqlin_dtype yt) {
+  constexpr int RP = F_ROWS / CS;                    // weight rows this CTA gathers and converts
+  constexpr int RPW = RP / F_PROD_WARPS;             // of which each producer warp owns
+  constexpr int LPR = 32 / RPW;                      // lanes per row
+  constexpr int SPT = 8 / LPR;                       // sub-vectors per lane and K-block
+  constexpr uint32_t PART_BYTES = RP * 128;          // this CTA's rows of a slot
+  static_assert(CS == 2 || CS == 4, "a cluster of 2 or 4 CTAs");
+  static_assert(RPW * LPR == 32 && SPT * LPR == 8, "producer lane map");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* ring_a = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* ring_b = ring_a + (size_t)FA_STAGES * FA_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(ring_b + (size_t)FB_STAGES * FB_BYTES);
-  uint64_t* a_full = bars;                          // [FA_STAGES], 8 producer-warp arrivals
-  uint64_t* a_empty = bars + FA_STAGES;             // [FA_STAGES], one commit
-  uint64_t* b_full = bars + 2 * FA_STAGES;          // [FB_STAGES], TMA transaction bytes
-  uint64_t* b_empty = b_full + FB_STAGES;           // [FB_STAGES], one commit
+  uint64_t* a_full = bars;                          // [FA_STAGES] the copier's arrival + peers' bytes
+  uint64_t* a_free = bars + FA_STAGES;              // [FA_STAGES] the MMA commit of every cluster CTA
+  uint64_t* own_full = bars + 2 * FA_STAGES;        // [FA_STAGES] this CTA's producer warps
+  uint64_t* b_full = bars + 3 * FA_STAGES;          // [FB_STAGES] TMA transaction bytes
+  uint64_t* b_empty = b_full + FB_STAGES;           // [FB_STAGES] one commit
   uint64_t* acc_bar = b_empty + FB_STAGES;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * F_ROWS;
-  const int64_t m0 = (int64_t)blockIdx.y * F_XROWS;
+  const int n0 = blockIdx.y * F_ROWS;               // weight rows of the cluster
+  const int64_t m0 = (int64_t)blockIdx.x * F_XROWS;
+  const uint32_t crank = cluster_rank();
   const int K = L.n_in;
   const int num_kb = (K + 63) / 64;
-  const int halves = (M - m0) > 256 ? 2 : 1;        // activation half-tiles of this CTA
+  const int halves = M - m0 > 256 ? 2 : (M - m0 > 0 ? 1 : 0);   // activation half-tiles of this CTA
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < FA_STAGES; ++s) {
-      mbar_init(smem_u32(&a_full[s]), F_PROD_WARPS);
-      mbar_init(smem_u32(&a_empty[s]), 1);
+      mbar_init(smem_u32(&a_full[s]), 1);
+      mbar_init(smem_u32(&a_free[s]), CS);
+      mbar_init(smem_u32(&own_full[s]), F_PROD_WARPS);
     }
     for (int s = 0; s < FB_STAGES; ++s) {
       mbar_init(smem_u32(&b_full[s]), 1);
@@ -396,6 +431,7 @@ __global__ void __launch_bounds__(F_THREADS, 1)
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
+  cluster_sync();                                  // every peer's barriers exist before any remote use
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = *tmem_holder;
   const int total_h = num_kb * halves;
@@ -414,7 +450,7 @@ __global__ void __launch_bounds__(F_THREADS, 1)
       issued_b = hk + 1;
     }
   } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer
+    // ---------------- MMA issuer (a CTA without activation rows still returns every slot)
     constexpr uint32_t idesc = idesc_f16(128, 256);
     int hk = 0;
     for (int kb = 0; kb < num_kb && !*abort_flag; ++kb) {
@@ -432,119 +468,204 @@ __global__ void __launch_bounds__(F_THREADS, 1)
         mma_commit(smem_u32(&b_empty[sb]));
       }
       if (*abort_flag) break;
-      mma_commit(smem_u32(&a_empty[sa]));
+      // the slot is free here once this MMA group completes: tell every CTA of the cluster
+      asm volatile(
+          "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+          ::"r"(smem_u32(&a_free[sa])), "h"((uint16_t)((1u << CS) - 1u)) : "memory");
     }
     mma_commit(smem_u32(acc_bar));
-  } else if (warp >= 2) {
-    // ---------------- weight producers
-    const int p = threadIdx.x - 64;
-    const int r = p & (F_ROWS - 1), hs = p >> 7;
+  } else if (warp == 2) {
+    // ---------------- copier: this CTA's rows of each K-block into every peer's slot
+    if (lane == 0) {
+      for (int kb = 0; kb < num_kb; ++kb) {
+        const int sa = kb % FA_STAGES;
+        if (*abort_flag || !mbar_wait(smem_u32(&own_full[sa]), (uint32_t)(kb / FA_STAGES) & 1u, 6)) {
+          *abort_flag = 1;
+          break;
+        }
+        const uint32_t full = smem_u32(&a_full[sa]);
+        const uint32_t part = smem_u32(ring_a + (size_t)sa * FA_BYTES) + crank * PART_BYTES;
+#pragma unroll
+        for (int q = 1; q < CS; ++q) {
+          const uint32_t peer = (crank + (uint32_t)q) % CS;
+          asm volatile(
+              "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+              ::"r"(peer_addr(part, peer)), "r"(part), "r"(PART_BYTES), "r"(peer_addr(full, peer))
+              : "memory");
+        }
+        mbar_expect_tx(full, (CS - 1) * PART_BYTES);   // this CTA's rows are in; the peers' are due
+      }
+    }
+  } else if (warp >= 3) {
+    // ---------------- weight producers: rows crank * RP + pw * RPW .. +RPW-1 of the tile
+    const int pw = warp - 3;
+    const int jg = lane % LPR;                        // sub-vectors jg * SPT .. +SPT-1 of a K-block
+    const int r = (int)crank * RP + pw * RPW + lane / LPR;   // row inside the 128-row tile
     const int64_t row = (int64_t)n0 + r;
     const bool row_ok = row < L.n_out;
     const uint8_t* codes_row = L.codes + (row_ok ? row : 0) * L.stride;
     const uint32_t m1 = (1u << L.bits1) - 1u;
     const float rsc = (L.rs && row_ok) ? __half2float(L.rs[row]) : 1.f;
     const bool has_cs = L.cs != nullptr;
-    int e = 0, e_end = 0;                              // this row's CSR entries not yet placed
-    if (L.nnz > 0 && row_ok) { e = L.row_ptr[row]; e_end = L.row_ptr[row + 1]; }
-    const uint32_t rsw = (uint32_t)(r & 7);
-    int next_j = e < e_end ? L.col[e] : 0x7FFFFFFF;     // column of the next CSR entry (prefetched)
-    int vb = 0, vb_end = 0;                             // this row's VSR blocks not yet placed
-    if (L.vsr_nb > 0 && row_ok) { vb = L.vsr_rp[row]; vb_end = L.vsr_rp[row + 1]; }
-    int next_s = vb < vb_end ? L.vsr_pos[vb] : 0x7FFFFFFF;   // sub-vector of the next VSR block
-    // issue the gathers of K-block kb into its slot (the slot must have been released by the MMA);
-    // false if the wait gave up (the whole warp then leaves together)
-    auto issue = [&](int kb) -> bool {
-      const int sa = kb % FA_STAGES;
-      const bool mine = !*abort_flag && mbar_wait(smem_u32(&a_empty[sa]), ((uint32_t)(kb / FA_STAGES) & 1u) ^ 1u, 3);
-      if (!__all_sync(0xffffffffu, mine)) { *abort_flag = 1; return false; }
-      const uint32_t slot = smem_u32(ring_a + (size_t)sa * FA_BYTES) + (uint32_t)r * 128u;
-      uint32_t fl[4];
-      if (row_ok) load_fields4<W>(codes_row, kb, hs, L.w, fl);   // the row's stride pads it past the last field
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int sl = 4 * hs + u, sv = kb * 8 + sl;
-        const uint32_t dst = slot + (((uint32_t)sl ^ rsw) << 4);
-        if (row_ok && sv < L.n_sub) {
-          const uint32_t f = (uint32_t)group_of(L, sv) * (uint32_t)L.k1 + (fl[u] & m1);
-          cp_async16(dst, reinterpret_cast<const uint4*>(L.cb1) + f);
-        } else {
-          asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
-        }
+    const int cbeg = jg * SPT * 8;                    // this lane's columns inside a K-block
+    // Every global load the producer needs is issued ahead of its use: index fields three steps
+    // before their gathers, centroids and column scales three K-blocks before their conversion,
+    // the CSR entries a chunk of four ahead and the VSR cursor two blocks ahead.
+    //
+    // A lane walks every CSR entry of its row in chunks of four entries aligned to four in the
+    // CSR arrays (one 16-byte load of columns, one 8-byte load of values; entries outside the row
+    // are skipped).  The chunk after the current one is loaded when the current one is entered, so
+    // no step waits on a load it has just issued.  (The chunks stay inside the arrays' 16 bytes of
+    // padding.)
+    int e_end = 0, cb = 0, ci = 0;                     // row end, current chunk, position in it
+    if (L.nnz > 0 && row_ok) {
+      const int e_beg = L.row_ptr[row];
+      e_end = L.row_ptr[row + 1];
+      cb = e_beg & ~3;
+      ci = e_beg - cb;
+    }
+    const int4* col4 = reinterpret_cast<const int4*>(L.col);
+    const uint2* val4 = reinterpret_cast<const uint2*>(L.val);
+    int4 cc = make_int4(0, 0, 0, 0), nc = cc;          // columns of the current and the next chunk
+    uint2 cv = make_uint2(0, 0), nv = cv;              // and their values
+    if (cb < e_end) { cc = __ldg(col4 + (cb >> 2)); cv = __ldg(val4 + (cb >> 2)); }
+    if (cb + 4 < e_end) { nc = __ldg(col4 + (cb >> 2) + 1); nv = __ldg(val4 + (cb >> 2) + 1); }
+    auto csr_col = [&]() -> int {
+      const int c = ci == 0 ? cc.x : ci == 1 ? cc.y : ci == 2 ? cc.z : cc.w;
+      return cb + ci < e_end ? c : 0x7FFFFFFF;
+    };
+    auto csr_val = [&]() -> uint16_t {
+      const uint32_t w = ci < 2 ? cv.x : cv.y;
+      return (uint16_t)((ci & 1) ? (w >> 16) : (w & 0xFFFFu));
+    };
+    auto csr_next = [&]() {
+      if (++ci == 4) {
+        ci = 0;
+        cb += 4;
+        cc = nc;
+        cv = nv;
+        if (cb + 4 < e_end) { nc = __ldg(col4 + (cb >> 2) + 1); nv = __ldg(val4 + (cb >> 2) + 1); }
       }
-      return true;
+    };
+    int vb = 0, vb_end = 0;                            // this row's VSR blocks not yet loaded
+    if (L.vsr_nb > 0 && row_ok) { vb = L.vsr_rp[row]; vb_end = L.vsr_rp[row + 1]; }
+    const uint4* vsr4 = reinterpret_cast<const uint4*>(L.vsr_val);
+    const uint4 z4 = make_uint4(0, 0, 0, 0);
+    int s0 = vb < vb_end ? L.vsr_pos[vb] : 0x7FFFFFFF;     // sub-vectors of the next two VSR blocks
+    uint4 b0 = vb < vb_end ? __ldg(vsr4 + vb) : z4;
+    ++vb;
+    int s1 = vb < vb_end ? L.vsr_pos[vb] : 0x7FFFFFFF;
+    uint4 b1 = vb < vb_end ? __ldg(vsr4 + vb) : z4;
+    ++vb;
+    const uint32_t rsw = (uint32_t)(r & 7);
+    const uint4* cb1v = reinterpret_cast<const uint4*>(L.cb1);
+    auto load_f = [&](int kb, uint32_t* f) {
+      if (row_ok && kb < num_kb) load_fields<W, SPT>(codes_row, kb, jg, L.w, L.n_sub, f);
+      else for (int u = 0; u < SPT; ++u) f[u] = 0u;
+    };
+    auto load_cs = [&](int kb, uint4* c) {
+#pragma unroll
+      for (int u = 0; u < SPT; ++u)
+        c[u] = (has_cs && row_ok && kb < num_kb && kb * 8 + SPT * jg + u < L.n_sub)
+                   ? __ldg(reinterpret_cast<const uint4*>(L.cs + kb * 64 + cbeg + u * 8)) : z4;
+    };
+    auto gather = [&](int kb, const uint32_t* fl, uint4* g) {
+#pragma unroll
+      for (int u = 0; u < SPT; ++u) {
+        const int sv = kb * 8 + SPT * jg + u;
+        if (row_ok && kb < num_kb && sv < L.n_sub)
+          g[u] = ldg_nc_na(cb1v + (uint32_t)group_of(L, sv) * (uint32_t)L.k1 + (fl[u] & m1));
+      }
     };
     bool ok = true;
-    // K-blocks 0 .. F_LOOKAHEAD - 1 first: their slots are free from the start
-    for (int kb = 0; kb < F_LOOKAHEAD; ++kb) {
-      if (ok && kb < num_kb) ok = issue(kb);
-      cp_async_commit();                                  // one group per K-block (possibly empty)
-    }
-    for (int kb = 0; kb < num_kb && ok; ++kb) {
-      // convert K-block kb in place as soon as this thread's copies have landed, so the MMA can
-      // take it while the gathers of the next K-blocks are still in flight
-      cp_async_wait<F_LOOKAHEAD - 1>();
+    // One pipeline step for K-block kb: the loads for later K-blocks; the conversion of kb into
+    // registers, with the VSR blocks of the lane's sub-vectors put in their places; then, once
+    // every CTA's MMA is done with kb's slot, the stores, the CSR values over them and the
+    // arrival for the copier.  The callers rotate fixed register arrays through the roles, so no value in
+    // flight is ever copied.
+    auto step = [&](int kb, const uint4* g_cur, uint4* g_next, const uint32_t* f_next, uint32_t* f_load,
+                    const uint4* c_cur, uint4* c_load) {
+      load_f(kb + 6, f_load);
+      load_cs(kb + 3, c_load);
+      gather(kb + 3, f_next, g_next);
+      uint32_t w4[SPT][4];
+#pragma unroll
+      for (int u = 0; u < SPT; ++u) {
+        const int sv = kb * 8 + SPT * jg + u;
+        w4[u][0] = w4[u][1] = w4[u][2] = w4[u][3] = 0u;
+        if (row_ok && sv < L.n_sub) {
+          const uint32_t cw[4] = {g_cur[u].x, g_cur[u].y, g_cur[u].z, g_cur[u].w};
+          const __half* ch = reinterpret_cast<const __half*>(&c_cur[u]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const __half2 h2 = *reinterpret_cast<const __half2*>(&cw[q]);
+            float a0 = __low2float(h2) * rsc, a1 = __high2float(h2) * rsc;   // exact
+            if (has_cs) {
+              a0 = rto_mul_f32(a0, __half2float(ch[2 * q]));
+              a1 = rto_mul_f32(a1, __half2float(ch[2 * q + 1]));
+            }
+            w4[u][q] = (uint32_t)__half_as_ushort(__float2half_rn(a0)) |
+                       ((uint32_t)__half_as_ushort(__float2half_rn(a1)) << 16);
+          }
+        }
+      }
+      const int col0 = kb * 64 + cbeg;                    // first column of this lane's sub-vectors
+      // VSR blocks of this row among the lane's sub-vectors replace them whole
+      while (s0 < kb * 8 + SPT * jg + SPT) {
+        const int u0 = s0 - (kb * 8 + SPT * jg);
+#pragma unroll
+        for (int u = 0; u < SPT; ++u)
+          if (u == u0) { w4[u][0] = b0.x; w4[u][1] = b0.y; w4[u][2] = b0.z; w4[u][3] = b0.w; }
+        s0 = s1; b0 = b1;
+        s1 = vb < vb_end ? L.vsr_pos[vb] : 0x7FFFFFFF;
+        b1 = vb < vb_end ? __ldg(vsr4 + vb) : z4;
+        ++vb;
+      }
+      // the slot is free once every CTA's MMA is done with its previous K-block
       const int sa = kb % FA_STAGES;
-      const uint32_t slot = smem_u32(ring_a + (size_t)sa * FA_BYTES) + (uint32_t)r * 128u;
-      const int col0 = kb * 64 + hs * 32;                 // first column of this thread's 4 sub-vectors
+      const bool mine = !*abort_flag && mbar_wait(smem_u32(&a_free[sa]), ((uint32_t)(kb / FA_STAGES) & 1u) ^ 1u, 3);
+      if (!__all_sync(0xffffffffu, mine)) { *abort_flag = 1; ok = false; return; }
+      const uint32_t slot0 = smem_u32(ring_a + (size_t)sa * FA_BYTES);
+      const uint32_t slot = slot0 + (uint32_t)r * 128u;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int sl = 4 * hs + u, sv = kb * 8 + sl;
-        if (!row_ok || sv >= L.n_sub) continue;
-        const uint32_t adr = slot + (((uint32_t)sl ^ rsw) << 4);
-        uint32_t w4[4];
-        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(w4[0]), "=r"(w4[1]), "=r"(w4[2]), "=r"(w4[3]) : "r"(adr));
-        float cj[8];
-        if (has_cs) {
-          const uint4 cu = __ldg(reinterpret_cast<const uint4*>(L.cs + col0 + u * 8));
-          const __half* ch = reinterpret_cast<const __half*>(&cu);
-#pragma unroll
-          for (int t = 0; t < 8; ++t) cj[t] = __half2float(ch[t]);
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const __half2 h2 = *reinterpret_cast<const __half2*>(&w4[q]);
-          float a0 = __low2float(h2) * rsc, a1 = __high2float(h2) * rsc;   // exact
-          if (has_cs) { a0 = rto_mul_f32(a0, cj[2 * q]); a1 = rto_mul_f32(a1, cj[2 * q + 1]); }
-          w4[q] = (uint32_t)__half_as_ushort(__float2half_rn(a0)) |
-                  ((uint32_t)__half_as_ushort(__float2half_rn(a1)) << 16);
-        }
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(adr), "r"(w4[0]), "r"(w4[1]), "r"(w4[2]),
-                     "r"(w4[3])
+      for (int u = 0; u < SPT; ++u) {
+        const uint32_t adr = slot + (((uint32_t)(SPT * jg + u) ^ rsw) << 4);
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(adr), "r"(w4[u][0]), "r"(w4[u][1]),
+                     "r"(w4[u][2]), "r"(w4[u][3])
                      : "memory");
       }
-      // sparse positions of this row inside the thread's 32 columns take the stored value
-      while (next_j < col0 + 32) {
-        if (next_j >= col0) {
-          const int k = next_j - kb * 64;                 // column inside the K-block
+      // sparse positions of this row inside the lane's columns take the stored value
+      for (int j = csr_col(); j < col0 + SPT * 8; j = csr_col()) {
+        if (j >= col0) {
+          const int k = j - kb * 64;                      // column inside the K-block
           const uint32_t adr = slot + ((((uint32_t)k >> 3) ^ rsw) << 4) + (((uint32_t)k & 7u) << 1);
-          asm volatile("st.shared.u16 [%0], %1;" ::"r"(adr), "h"(L.val[e]) : "memory");
+          asm volatile("st.shared.u16 [%0], %1;" ::"r"(adr), "h"(csr_val()) : "memory");
         }
-        ++e;
-        next_j = e < e_end ? L.col[e] : 0x7FFFFFFF;
-      }
-      // VSR blocks of this row among the thread's 4 sub-vectors replace them whole (16 bytes)
-      while (next_s < kb * 8 + 4 * hs + 4) {
-        if (next_s >= kb * 8 + 4 * hs) {
-          const uint4 v = __ldg(reinterpret_cast<const uint4*>(L.vsr_val) + vb);
-          const uint32_t adr = slot + (((uint32_t)(next_s - kb * 8) ^ rsw) << 4);
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(adr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-                       : "memory");
-        }
-        ++vb;
-        next_s = vb < vb_end ? L.vsr_pos[vb] : 0x7FFFFFFF;
+        csr_next();
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
-      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&a_full[sa])) : "memory");
-      // then refill: the gathers of K-block kb + F_LOOKAHEAD go to the slot of K-block kb - 1
-      if (kb + F_LOOKAHEAD < num_kb) ok = issue(kb + F_LOOKAHEAD);
-      cp_async_commit();
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&own_full[sa])) : "memory");
+    };
+    // Array X_i holds the values of K-blocks congruent to i mod 4.
+    uint4 G0[SPT], G1[SPT], G2[SPT], G3[SPT];          // centroids in flight
+    uint32_t F0[SPT], F1[SPT], F2[SPT], F3[SPT];       // index fields
+    uint4 C0[SPT], C1[SPT], C2[SPT], C3[SPT];          // column scales
+    load_f(0, F0); load_f(1, F1); load_f(2, F2); load_f(3, F3);
+    gather(0, F0, G0); gather(1, F1, G1); gather(2, F2, G2);
+    load_f(4, F0); load_f(5, F1);
+    load_cs(0, C0); load_cs(1, C1); load_cs(2, C2);
+    for (int kb = 0; kb < num_kb && ok; kb += 4) {
+      step(kb, G0, G3, F3, F2, C0, C3);
+      if (!ok || kb + 1 >= num_kb) break;
+      step(kb + 1, G1, G0, F0, F3, C1, C0);
+      if (!ok || kb + 2 >= num_kb) break;
+      step(kb + 2, G2, G1, F1, F0, C2, C1);
+      if (!ok || kb + 3 >= num_kb) break;
+      step(kb + 3, G3, G2, F2, F1, C3, C2);
     }
-    cp_async_wait<0>();                                   // nothing of ours may land after exit
-    // ---------------- epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31, accumulator (w - 2) / 4
-    const int q = warp & 3, half = (warp - 2) >> 2;
+    // ---------------- epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31, accumulator (w - 3) / 4
+    const int q = warp & 3, half = (warp - 3) >> 2;
     const bool done = mbar_wait(smem_u32(acc_bar), 0, 4);
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     // tcgen05.ld is warp-wide: the whole warp reads, or none of it
@@ -558,9 +679,9 @@ __global__ void __launch_bounds__(F_THREADS, 1)
         const int64_t mb = m0 + half * 256 + c;
         if (!i_ok) continue;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int64_t m = mb + j;
-          if (m < M) store_from_float(Y, yt, m * L.n_out + i, __uint_as_float(v[j]));
+        for (int jx = 0; jx < 32; ++jx) {
+          const int64_t m = mb + jx;
+          if (m < M) store_from_float(Y, yt, m * L.n_out + i, __uint_as_float(v[jx]));
         }
       }
     }
@@ -577,6 +698,15 @@ __global__ void __launch_bounds__(F_THREADS, 1)
     __syncwarp();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512) : "memory");
+  }
+  // Every copy and slot release into this CTA was issued before its sender reached this barrier.
+  // On the normal path each copy has landed (this CTA's MMA consumed every K-block); after an
+  // abort give the ones still in flight (a few KB, microseconds) time to land before the CTA exits.
+  __syncwarp();
+  cluster_sync();
+  if (*abort_flag) {
+    const uint64_t t0 = now_ns();
+    while (now_ns() - t0 < 100000ull) __nanosleep(1000);
   }
 }
 
@@ -633,18 +763,42 @@ bool gemm_fused_supported(const Layer& L) {
   return L.d == 8 && L.k2 == 0 && L.n_ocols == 0 && L.n_sub > 0 && (L.n_in % 8) == 0 && L.w <= 32;
 }
 
+template <int CS>
+static cudaError_t launch_vq_cs(const Layer& L, const CUtensorMap& mx, int64_t M, void* Y, vqlin_dtype yt,
+                                cudaStream_t s) {
+  auto k = L.w == 8 ? tc::k_gemm_vq<8, CS> : L.w == 16 ? tc::k_gemm_vq<16, CS> : L.w == 32 ? tc::k_gemm_vq<32, CS>
+                                                                                           : tc::k_gemm_vq<0, CS>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::F_SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  // activation groups on x (rounded up to whole clusters: a CTA past M only gathers and shares
+  // its rows), weight tiles on y
+  const int64_t groups = (M + tc::F_XROWS - 1) / tc::F_XROWS;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3((unsigned)((groups + CS - 1) / CS * CS), (unsigned)((L.n_out + tc::F_ROWS - 1) / tc::F_ROWS));
+  cfg.blockDim = dim3(tc::F_THREADS);
+  cfg.dynamicSmemBytes = tc::F_SMEM_BYTES;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  note_launches(1);
+  return cudaLaunchKernelEx(&cfg, k, mx, L, M, Y, yt);
+}
+
 cudaError_t launch_gemm_vq(const Layer& L, const __half* X, int64_t M, void* Y, vqlin_dtype yt, cudaStream_t s) {
   if (!gemm_fused_supported(L) || (reinterpret_cast<uintptr_t>(X) & 15) || M < 1 || M > 0x7FFFFFFF)
     return cudaErrorInvalidValue;
   CUtensorMap mx;
   if (!make_map(&mx, X, (uint64_t)M, (uint64_t)L.n_in, 256)) return cudaErrorInvalidValue;
-  auto k = L.w == 8 ? tc::k_gemm_vq<8> : L.w == 12 ? tc::k_gemm_vq<12> : L.w == 16 ? tc::k_gemm_vq<16>
-         : L.w == 24 ? tc::k_gemm_vq<24> : L.w == 32 ? tc::k_gemm_vq<32> : tc::k_gemm_vq<0>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::F_SMEM_BYTES);
+  // A cluster shares each weight tile over four 512-row activation groups, or two up to 1024
+  // activation rows (a CTA past the last row still converts and shares its part of the tile).
+  const int64_t groups = (M + tc::F_XROWS - 1) / tc::F_XROWS;
+  cudaError_t e = groups > 2 ? launch_vq_cs<4>(L, mx, M, Y, yt, s) : launch_vq_cs<2>(L, mx, M, Y, yt, s);
   if (e != cudaSuccess) return e;
-  dim3 grid((L.n_out + tc::F_ROWS - 1) / tc::F_ROWS, (unsigned)((M + tc::F_XROWS - 1) / tc::F_XROWS));
-  note_launches(1);
-  k<<<grid, tc::F_THREADS, tc::F_SMEM_BYTES, s>>>(mx, L, M, Y, yt);
   return cudaGetLastError();
 }
 

@@ -289,12 +289,14 @@ def test_gemm_small(vq, t, M):
     G.assert_close(Y, oracle.gemv_f64(L, synth.bits_to_f64(Xb, "bf16")), "f32", "gemm small")
 
 
-@pytest.mark.parametrize("M", [1, 300, 513, 1100])
+@pytest.mark.parametrize("M", [1, 300, 513, 1100, 1600, 2100])
 def test_gemm_fused_ragged_tiles(vq, M):
     """The fused prefill (weight tiles dequantised in shared memory): 300 weight rows (three
     128-row tiles, the last ragged), 200 columns (three whole K-blocks and a partial one), row and
-    column scales and CSR replacements; M covers one and two activation halves and several
-    512-row groups."""
+    column scales and CSR replacements; M covers one and two activation halves and one to five
+    512-row groups, so clusters of 2 and 4 CTAs sharing each weight tile, with CTAs past the last
+    activation row (1 and 300: one group in a cluster of 2; 1100: 3 groups in a cluster of 4;
+    2100: 5 groups in 2 clusters of 4)."""
     import torch
     rng = np.random.default_rng(4300 + M)
     L = synth.random_layer(rng, 300, 200, 8, 256, 8, col_scale=True, cb_std=0.3, nnz=700, outlier_scale=1.0)
@@ -306,6 +308,24 @@ def test_gemm_fused_ragged_tiles(vq, M):
     torch.cuda.synchronize()
     assert vq.device_error() == 0
     G.assert_close(G.to_f64(Y), oracle.gemv_f64(L, synth.bits_to_f64(Xb, "f16")), "f32", "fused gemm M=%d" % M)
+
+
+@pytest.mark.parametrize("t", [13, 14, 15, 19])
+@pytest.mark.parametrize("M", [1100, 2100])
+def test_gemm_fused_cluster_formats(vq, t, M):
+    """VSR blocks, codebook groups and the symmetric codebook through the fused prefill when
+    2 and 4 CTAs share each weight tile (each dequantises a part of the tile's rows)."""
+    import torch
+    L = SMALL[t]
+    rng = np.random.default_rng(4400 + M + t)
+    Xb = synth.activations(rng, M, L.n_in, "f16")
+    m = vq.VQLinear(L)
+    n0 = vq.vqlin_kernel_launches()
+    Y = m.gemm(G.torch_x(Xb, "f16"), out_dtype=torch.float32)
+    assert vq.vqlin_kernel_launches() - n0 == 1
+    torch.cuda.synchronize()
+    assert vq.device_error() == 0
+    G.assert_close(G.to_f64(Y), oracle.gemv_f64(L, synth.bits_to_f64(Xb, "f16")), "f32", "fused gemm t=%d M=%d" % (t, M))
 
 
 def test_gemm_prefill_sampled_rows(vq):
