@@ -625,6 +625,25 @@ vqlin_status vqlin_create(const vqlin_desc* D, void* stream, vqlin_handle** out)
     L.vsr_val = up.put<uint16_t>(vvals.data(), vvals.size());
     L.vsr_delta = up.put<float>(vdelta.data(), vdelta.size() * 4);
   }
+  if (D->nnz && gemm_fused_supported(L)) {
+    // the CSR entries by 64-column K-block for the fused prefill GEMM
+    const int32_t nkb = (D->n_in + 63) / 64;
+    std::vector<int32_t> kbs((size_t)D->n_out * (nkb + 1));
+    std::vector<uint32_t> kbe((size_t)D->nnz);
+    const int32_t* r = as<int32_t>(rp);
+    const int32_t* c = as<int32_t>(ci);
+    const uint16_t* v = as<uint16_t>(vals);
+    for (int32_t i = 0; i < D->n_out; ++i) {
+      int32_t e = r[i];
+      for (int32_t kb = 0; kb <= nkb; ++kb) {
+        while (e < r[i + 1] && c[e] < kb * 64) ++e;
+        kbs[(size_t)i * (nkb + 1) + kb] = e;
+      }
+    }
+    for (int64_t e = 0; e < D->nnz; ++e) kbe[e] = ((uint32_t)(c[e] & 63) << 16) | v[e];
+    L.kb_start = up.put<int32_t>(kbs.data(), kbs.size() * 4);
+    L.kb_entry = up.put<uint32_t>(kbe.data(), kbe.size() * 4);
+  }
   L.tcodes = tcodes.empty() ? nullptr : up.put<uint8_t>(tcodes.data(), tcodes.size());
   if (!cs_words.empty()) {
     L.cs_words = up.put<uint64_t>(cs_words.data(), cs_words.size() * 8);

@@ -273,34 +273,34 @@ __global__ void __launch_bounds__(THREADS, 1)
 //
 // Sharing the weight tile.  The CS CTAs of a thread-block cluster (CS = 2 up to 1024 activation
 // rows, 4 beyond) own the same 128 weight rows and different 512-row activation groups (a CTA past
-// the last activation row still converts and shares its part).  Each gathers and
-// converts only its 128 / CS rows of every weight K-block into its own slot, and one thread copies
-// them into the same slot of each peer (cp.async.bulk shared::cta -> shared::cluster, completing
-// on the peer's slot barrier).  So every weight element is gathered
-// and converted once per 512 * CS activation rows.  A slot is rewritten only when every CTA's MMA
-// has finished with it: the MMA returns a slot with one tcgen05.commit multicast to the slot's
-// "cluster empty" barrier in every CTA of the cluster.
+// the last activation row still converts and shares its part).  Each converts only its 128 / CS
+// rows of every weight K-block into its own slot, and one thread copies them into the same slot
+// of each peer (cp.async.bulk shared::cta -> shared::cluster, completing on the peer's slot
+// barrier).  So every weight element is gathered and converted once per 512 * CS activation rows.
+// A slot is rewritten only when every CTA's MMA has finished with it: the MMA returns a slot with
+// one tcgen05.commit multicast to the slot's "cluster free" barrier in every CTA of the cluster.
 //
-// Warp roles (11 warps):
+// Warp roles (18 + 128 / (32 CS) warps):
 //   warp 0      TMA producer of the activation tiles: 256 rows x 64 k (one 128-byte swizzle row
 //               per activation row) into a 5-slot ring of half K-blocks;
 //   warp 1      allocates the 512 TMEM columns; one lane issues tcgen05.mma.kind::f16 (M = 128,
 //               N = 256, K = 16), four per half K-block, and returns ring slots with
 //               tcgen05.commit;
-//   warp 2      one lane copies this CTA's rows of each weight K-block to the peers once its
-//               producers have written them, and arms the slot's full barrier for the peers' bytes;
-//   warps 3-10  weight producers, then the epilogue.  A producer warp owns 16 / CS consecutive
-//               rows of this CTA's part (128 / CS rows); 2 CS lanes share a row, each with 4 / CS
-//               of the row's 8 sub-vectors in a K-block (64 columns).  Three K-blocks ahead a lane
-//               gathers its centroids into registers (index fields loaded two steps earlier
-//               still).  For K-block kb it converts them to the exact fp16 weight
-//               fp16(r_i c_j C[k][t]) (C r_i is exact in fp32; the product with c_j is rounded to
-//               odd in fp32, so the final fp16 rounding is the correctly rounded one, as in the
-//               exact dequantisation) and puts the VSR blocks of its sub-vectors in their places
-//               (REPLACE), all while the slot may still be in use.  Once the slot is free it stores
-//               them to their 128-byte-swizzled places (chunk s ^ (row % 8) of the row's 128
-//               bytes, the layout a TMA 128B-swizzle load makes), writes the CSR values of its
-//               columns over them (REPLACE) and makes the writes visible to the async proxy
+//   sparse warps (one per 32 rows of this CTA's part) the sparse part: once the producers have
+//               written a K-block of this CTA's rows, a lane per row writes the row's CSR values
+//               and VSR blocks in that K-block over them (REPLACE); then one lane copies the warp's
+//               rows to the peers and arrives on the slot's full barrier (the first sparse warp
+//               also arms it for the peers' bytes);
+//   16 warps    weight producers, then the epilogue.  The 512 lanes cover this CTA's 128 / CS rows
+//               x 8 sub-vectors of a K-block (64 columns): a lane owns one sub-vector (CS = 2) or
+//               half of one (CS = 4).  Three K-blocks ahead a lane gathers its part of the
+//               centroid into registers (index fields loaded three steps before that).  For
+//               K-block kb it converts it to the exact fp16 weight fp16(r_i c_j C[k][t]) (C r_i is
+//               exact in fp32; the product with c_j is rounded to odd in fp32, so the final fp16
+//               rounding is the correctly rounded one, as in the exact dequantisation) while the
+//               slot may still be in use; once the slot is free it stores it to its
+//               128-byte-swizzled place (chunk s ^ (row % 8) of the row's 128 bytes, the layout a
+//               TMA 128B-swizzle load makes) and makes the writes visible to the async proxy
 //               (fence.proxy.async).  The weight tile is therefore bit for bit the dequantised W.
 // Every mbarrier wait is bounded (1 s); on expiry the kernel records an error code, stops,
 // waits (bounded) for its own copies, frees TMEM and returns.  Every thread reaches the cluster
@@ -308,8 +308,9 @@ __global__ void __launch_bounds__(THREADS, 1)
 constexpr int FA_STAGES = 4, FB_STAGES = 5;
 constexpr int FA_BYTES = 128 * 64 * 2;             // 16 KB weight slot
 constexpr int FB_BYTES = 256 * 64 * 2;             // 32 KB activation half-slot
-constexpr int F_PROD_WARPS = 8;
-constexpr int F_THREADS = (3 + F_PROD_WARPS) * 32;
+constexpr int F_PROD_WARPS = 16;
+// threads of the kernel for a cluster of cs CTAs: TMA, MMA, 4 / cs sparse warps, the producers
+__host__ __device__ constexpr int f_threads(int cs) { return (2 + 4 / cs + F_PROD_WARPS) * 32; }
 constexpr int F_ROWS = 128, F_XROWS = 512;
 constexpr size_t F_SMEM_BYTES = 1024 + (size_t)FA_STAGES * FA_BYTES + (size_t)FB_STAGES * FB_BYTES + 256;
 
@@ -346,52 +347,35 @@ __device__ __forceinline__ void cluster_sync() {
 }
 
 
-// The SPT index fields of sub-vectors kb*8 + SPT*j .. +SPT-1 of one packed row: SPT*w/8 bytes at
-// byte kb*w + j*SPT*w/8 (the eight fields of a K-block are w bytes).  One load when w is 8, 16 or
-// 32 (the row stride, a multiple of 16 bytes, and the 16 bytes of padding after the array cover
-// the K-block past the last sub-vector); field by field otherwise (W = 0: any width), fields at
-// or past n_sub reading as 0.
-template <int W, int SPT>
-__device__ __forceinline__ void load_fields(const uint8_t* row, int kb, int j, int w, int n_sub, uint32_t* f) {
-  constexpr int BYTES = SPT * W / 8;
-  const uint8_t* p = row + kb * W + j * BYTES;
-  if constexpr (W == 8 || W == 16 || W == 32) {
-    uint32_t v[SPT * W / 32 > 0 ? SPT * W / 32 : 1];
-    if constexpr (BYTES == 1) v[0] = __ldg(p);
-    else if constexpr (BYTES == 2) v[0] = __ldg(reinterpret_cast<const unsigned short*>(p));
-    else if constexpr (BYTES == 4) v[0] = __ldg(reinterpret_cast<const uint32_t*>(p));
-    else if constexpr (BYTES == 8) { const uint2 t = __ldg(reinterpret_cast<const uint2*>(p)); v[0] = t.x; v[1] = t.y; }
-    else { const uint4 t = __ldg(reinterpret_cast<const uint4*>(p)); v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w; }
-#pragma unroll
-    for (int u = 0; u < SPT; ++u) {
-      const int bit = u * W;
-      f[u] = W == 32 ? v[u] : (v[bit >> 5] >> (bit & 31)) & ((1u << (W & 31)) - 1u);
-    }
-  } else {
-#pragma unroll
-    for (int u = 0; u < SPT; ++u) {
-      const int sv = kb * 8 + SPT * j + u;
-      f[u] = sv < n_sub ? read_field(row, sv, w) : 0u;
-    }
-  }
+// The index field of sub-vector s of one packed row (W = 8, 16, 32: one aligned load; W = 0: any
+// width).
+template <int W>
+__device__ __forceinline__ uint32_t load_field(const uint8_t* row, int s, int w) {
+  if constexpr (W == 8) return __ldg(row + s);
+  else if constexpr (W == 16) return __ldg(reinterpret_cast<const unsigned short*>(row) + s);
+  else if constexpr (W == 32) return __ldg(reinterpret_cast<const uint32_t*>(row) + s);
+  else return read_field(row, s, w);
 }
 
 template <int W, int CS>
-__global__ void __launch_bounds__(F_THREADS, 1)
+__global__ void __launch_bounds__(f_threads(CS), 1)
     k_gemm_vq(const __grid_constant__ CUtensorMap map_x, const Layer L, int64_t M, void* __restrict__ Y,
               vqlin_dtype yt) {
-  constexpr int RP = F_ROWS / CS;                    // weight rows this CTA gathers and converts
-  constexpr int RPW = RP / F_PROD_WARPS;             // of which each producer warp owns
-  constexpr int LPR = 32 / RPW;                      // lanes per row
-  constexpr int SPT = 8 / LPR;                       // sub-vectors per lane and K-block
-  constexpr uint32_t PART_BYTES = RP * 128;          // this CTA's rows of a slot
   static_assert(CS == 2 || CS == 4, "a cluster of 2 or 4 CTAs");
-  static_assert(RPW * LPR == 32 && SPT * LPR == 8, "producer lane map");
+  constexpr int RP = F_ROWS / CS;                    // weight rows this CTA converts
+  constexpr int HS = CS / 2;                         // lanes per sub-vector
+  constexpr int NW = 4 / HS;                         // 32-bit words (fp16 pairs) per lane
+  constexpr int RPW = RP / F_PROD_WARPS;             // rows per producer warp
+  constexpr int LPR = 32 / RPW;                      // lanes per row
+  constexpr int NSP = RP / 32;                       // sparse warps, a row per lane
+  constexpr int PW0 = 2 + NSP;                       // first producer warp
+  constexpr uint32_t PART_BYTES = RP * 128;          // this CTA's rows of a slot
+  static_assert(LPR == 8 * HS && NSP >= 1, "lane map");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* ring_a = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* ring_b = ring_a + (size_t)FA_STAGES * FA_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(ring_b + (size_t)FB_STAGES * FB_BYTES);
-  uint64_t* a_full = bars;                          // [FA_STAGES] the copier's arrival + peers' bytes
+  uint64_t* a_full = bars;                          // [FA_STAGES] the sparse warps' arrivals + peers' bytes
   uint64_t* a_free = bars + FA_STAGES;              // [FA_STAGES] the MMA commit of every cluster CTA
   uint64_t* own_full = bars + 2 * FA_STAGES;        // [FA_STAGES] this CTA's producer warps
   uint64_t* b_full = bars + 3 * FA_STAGES;          // [FB_STAGES] TMA transaction bytes
@@ -410,7 +394,7 @@ __global__ void __launch_bounds__(F_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < FA_STAGES; ++s) {
-      mbar_init(smem_u32(&a_full[s]), 1);
+      mbar_init(smem_u32(&a_full[s]), NSP);
       mbar_init(smem_u32(&a_free[s]), CS);
       mbar_init(smem_u32(&own_full[s]), F_PROD_WARPS);
     }
@@ -474,32 +458,111 @@ __global__ void __launch_bounds__(F_THREADS, 1)
           ::"r"(smem_u32(&a_free[sa])), "h"((uint16_t)((1u << CS) - 1u)) : "memory");
     }
     mma_commit(smem_u32(acc_bar));
-  } else if (warp == 2) {
-    // ---------------- copier: this CTA's rows of each K-block into every peer's slot
-    if (lane == 0) {
-      for (int kb = 0; kb < num_kb; ++kb) {
-        const int sa = kb % FA_STAGES;
-        if (*abort_flag || !mbar_wait(smem_u32(&own_full[sa]), (uint32_t)(kb / FA_STAGES) & 1u, 6)) {
-          *abort_flag = 1;
-          break;
-        }
+  } else if (warp >= 2 && warp < PW0) {
+    // ---------------- sparse part and copies: lane l of sparse warp sw owns row
+    // crank * RP + 32 sw + l of the tile.  The row's CSR entries come by K-block: the start and end
+    // of K-block x four steps ahead, up to four of its entries (column in the block, value) two
+    // steps ahead, so the K-block's work is a few stores; more than four entries in one row and
+    // K-block (rare) are loaded on the spot.  The VSR blocks come two ahead.
+    const int sw = warp - 2;
+    const int rt = (int)crank * RP + sw * 32 + lane;
+    const int64_t row = (int64_t)n0 + rt;
+    const bool row_ok = row < L.n_out;
+    const bool has_csr = L.nnz > 0 && row_ok;
+    const int32_t* kbs = has_csr ? L.kb_start + row * (num_kb + 1) : nullptr;
+    const uint32_t* kbe = L.kb_entry;
+    const uint32_t slot_row = (uint32_t)rt * 128u, rsw = (uint32_t)(rt & 7);
+    int vb = 0, vb_end = 0;                          // VSR cursor, two blocks ahead
+    if (L.vsr_nb > 0 && row_ok) { vb = L.vsr_rp[row]; vb_end = L.vsr_rp[row + 1]; }
+    const uint4* vsr4 = reinterpret_cast<const uint4*>(L.vsr_val);
+    const uint4 z4 = make_uint4(0, 0, 0, 0);
+    int s0 = vb < vb_end ? L.vsr_pos[vb] : 0x7FFFFFFF;
+    uint4 b0 = vb < vb_end ? __ldg(vsr4 + vb) : z4;
+    ++vb;
+    int s1 = vb < vb_end ? L.vsr_pos[vb] : 0x7FFFFFFF;
+    uint4 b1 = vb < vb_end ? __ldg(vsr4 + vb) : z4;
+    ++vb;
+    struct Ent { uint32_t e[4]; int s, n; };
+    auto load_t = [&](int x, int2& t) {
+      if (has_csr) { x = min(x, num_kb - 1); t.x = __ldg(kbs + x); t.y = __ldg(kbs + x + 1); }
+      else t = make_int2(0, 0);
+    };
+    auto load_e = [&](const int2& t, Ent& en) {
+      en.s = t.x;
+      en.n = t.y - t.x;
+      if (en.n > 0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) en.e[i] = __ldg(kbe + t.x + i);   // inside the 16 bytes of padding
+      }
+    };
+    auto put = [&](uint32_t slot, uint32_t ent) {
+      const uint32_t k = ent >> 16;                   // column inside the K-block
+      const uint32_t adr = slot + ((((k >> 3) ^ rsw) << 4) | ((k & 7u) << 1));
+      asm volatile("st.shared.u16 [%0], %1;" ::"r"(adr), "h"((uint16_t)(ent & 0xFFFFu)) : "memory");
+    };
+    bool ok = true;
+    // K-block kb: the stores once the producers are done, then the copies; T and E rotate as in
+    // the producers (array i holds K-blocks congruent to i mod 4)
+    auto sstep = [&](int kb, int2& t_load, const int2& t_use, Ent& e_load, const Ent& e_cur) {
+      const int sa = kb % FA_STAGES;
+      const bool mine = !*abort_flag && mbar_wait(smem_u32(&own_full[sa]), (uint32_t)(kb / FA_STAGES) & 1u, 6);
+      if (!__all_sync(0xffffffffu, mine)) { *abort_flag = 1; ok = false; return; }
+      const uint32_t slot0 = smem_u32(ring_a + (size_t)sa * FA_BYTES);
+      const uint32_t slot = slot0 + slot_row;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (i < e_cur.n) put(slot, e_cur.e[i]);
+      for (int i = 4; i < e_cur.n; ++i) put(slot, __ldg(kbe + e_cur.s + i));
+      while (s0 < (kb + 1) * 8) {
+        const uint32_t adr = slot + (((uint32_t)(s0 - kb * 8) ^ rsw) << 4);
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(adr), "r"(b0.x), "r"(b0.y), "r"(b0.z),
+                     "r"(b0.w)
+                     : "memory");
+        s0 = s1;
+        b0 = b1;
+        s1 = vb < vb_end ? L.vsr_pos[vb] : 0x7FFFFFFF;
+        b1 = vb < vb_end ? __ldg(vsr4 + vb) : z4;
+        ++vb;
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) {
+        // the warp's rows of the K-block are complete: copy them into every peer's slot
         const uint32_t full = smem_u32(&a_full[sa]);
-        const uint32_t part = smem_u32(ring_a + (size_t)sa * FA_BYTES) + crank * PART_BYTES;
+        const uint32_t part = slot0 + (uint32_t)(crank * RP + sw * 32) * 128u;
 #pragma unroll
         for (int q = 1; q < CS; ++q) {
           const uint32_t peer = (crank + (uint32_t)q) % CS;
           asm volatile(
               "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-              ::"r"(peer_addr(part, peer)), "r"(part), "r"(PART_BYTES), "r"(peer_addr(full, peer))
+              ::"r"(peer_addr(part, peer)), "r"(part), "r"(32u * 128u), "r"(peer_addr(full, peer))
               : "memory");
         }
-        mbar_expect_tx(full, (CS - 1) * PART_BYTES);   // this CTA's rows are in; the peers' are due
+        if (sw == 0) mbar_expect_tx(full, (CS - 1) * PART_BYTES);   // the peers' rows are due
+        else asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(full) : "memory");
       }
+      load_e(t_use, e_load);
+      load_t(kb + 4, t_load);
+    };
+    int2 T0, T1, T2, T3;
+    Ent E0, E1, E2, E3;
+    load_t(0, T0); load_t(1, T1); load_t(2, T2); load_t(3, T3);
+    load_e(T0, E0); load_e(T1, E1);
+    E2.n = E3.n = 0;
+    for (int kb = 0; kb < num_kb && ok; kb += 4) {
+      sstep(kb, T0, T2, E2, E0);
+      if (!ok || kb + 1 >= num_kb) break;
+      sstep(kb + 1, T1, T3, E3, E1);
+      if (!ok || kb + 2 >= num_kb) break;
+      sstep(kb + 2, T2, T0, E0, E2);
+      if (!ok || kb + 3 >= num_kb) break;
+      sstep(kb + 3, T3, T1, E1, E3);
     }
-  } else if (warp >= 3) {
-    // ---------------- weight producers: rows crank * RP + pw * RPW .. +RPW-1 of the tile
-    const int pw = warp - 3;
-    const int jg = lane % LPR;                        // sub-vectors jg * SPT .. +SPT-1 of a K-block
+  } else if (warp >= PW0) {
+    // ---------------- weight producers
+    const int pw = warp - PW0;
+    const int it = lane % LPR;                        // item of the row: sub-vector it / HS, part it % HS
+    const int svl = it / HS, hp = it % HS;
     const int r = (int)crank * RP + pw * RPW + lane / LPR;   // row inside the 128-row tile
     const int64_t row = (int64_t)n0 + r;
     const bool row_ok = row < L.n_out;
@@ -507,153 +570,84 @@ __global__ void __launch_bounds__(F_THREADS, 1)
     const uint32_t m1 = (1u << L.bits1) - 1u;
     const float rsc = (L.rs && row_ok) ? __half2float(L.rs[row]) : 1.f;
     const bool has_cs = L.cs != nullptr;
-    const int cbeg = jg * SPT * 8;                    // this lane's columns inside a K-block
-    // Every global load the producer needs is issued ahead of its use: index fields three steps
-    // before their gathers, centroids and column scales three K-blocks before their conversion,
-    // the CSR entries a chunk of four ahead and the VSR cursor two blocks ahead.
-    //
-    // A lane walks every CSR entry of its row in chunks of four entries aligned to four in the
-    // CSR arrays (one 16-byte load of columns, one 8-byte load of values; entries outside the row
-    // are skipped).  The chunk after the current one is loaded when the current one is entered, so
-    // no step waits on a load it has just issued.  (The chunks stay inside the arrays' 16 bytes of
-    // padding.)
-    int e_end = 0, cb = 0, ci = 0;                     // row end, current chunk, position in it
-    if (L.nnz > 0 && row_ok) {
-      const int e_beg = L.row_ptr[row];
-      e_end = L.row_ptr[row + 1];
-      cb = e_beg & ~3;
-      ci = e_beg - cb;
-    }
-    const int4* col4 = reinterpret_cast<const int4*>(L.col);
-    const uint2* val4 = reinterpret_cast<const uint2*>(L.val);
-    int4 cc = make_int4(0, 0, 0, 0), nc = cc;          // columns of the current and the next chunk
-    uint2 cv = make_uint2(0, 0), nv = cv;              // and their values
-    if (cb < e_end) { cc = __ldg(col4 + (cb >> 2)); cv = __ldg(val4 + (cb >> 2)); }
-    if (cb + 4 < e_end) { nc = __ldg(col4 + (cb >> 2) + 1); nv = __ldg(val4 + (cb >> 2) + 1); }
-    auto csr_col = [&]() -> int {
-      const int c = ci == 0 ? cc.x : ci == 1 ? cc.y : ci == 2 ? cc.z : cc.w;
-      return cb + ci < e_end ? c : 0x7FFFFFFF;
+    const uint32_t rsw = (uint32_t)(r & 7);
+    const uint32_t* cb1w = reinterpret_cast<const uint32_t*>(L.cb1);
+    const int last_kb = num_kb - 1;
+    // Every global load is issued ahead of its use and unconditionally (K-block indices past the
+    // last are clamped; values for sub-vectors past the last are never used): index fields three
+    // steps before their gathers, centroids and column scales three K-blocks before their
+    // conversion.
+    auto load_f = [&](int kb) -> uint32_t {
+      return load_field<W>(codes_row, min(min(kb, last_kb) * 8 + svl, L.n_sub - 1), L.w);
     };
-    auto csr_val = [&]() -> uint16_t {
-      const uint32_t w = ci < 2 ? cv.x : cv.y;
-      return (uint16_t)((ci & 1) ? (w >> 16) : (w & 0xFFFFu));
-    };
-    auto csr_next = [&]() {
-      if (++ci == 4) {
-        ci = 0;
-        cb += 4;
-        cc = nc;
-        cv = nv;
-        if (cb + 4 < e_end) { nc = __ldg(col4 + (cb >> 2) + 1); nv = __ldg(val4 + (cb >> 2) + 1); }
+    auto load_cs = [&](int kb, uint32_t* c) {
+      // the 8 / HS column scales of the lane's part (clamped into the vector: unused past n_in)
+      const int col = min(min(kb, last_kb) * 64 + svl * 8 + hp * (8 / HS), K - 8 / HS);
+      if constexpr (NW == 4) {
+        const uint4 t = has_cs ? __ldg(reinterpret_cast<const uint4*>(L.cs + col)) : make_uint4(0, 0, 0, 0);
+        c[0] = t.x; c[1] = t.y; c[2] = t.z; c[3] = t.w;
+      } else {
+        const uint2 t = has_cs ? __ldg(reinterpret_cast<const uint2*>(L.cs + col)) : make_uint2(0, 0);
+        c[0] = t.x; c[1] = t.y;
       }
     };
-    int vb = 0, vb_end = 0;                            // this row's VSR blocks not yet loaded
-    if (L.vsr_nb > 0 && row_ok) { vb = L.vsr_rp[row]; vb_end = L.vsr_rp[row + 1]; }
-    const uint4* vsr4 = reinterpret_cast<const uint4*>(L.vsr_val);
-    const uint4 z4 = make_uint4(0, 0, 0, 0);
-    int s0 = vb < vb_end ? L.vsr_pos[vb] : 0x7FFFFFFF;     // sub-vectors of the next two VSR blocks
-    uint4 b0 = vb < vb_end ? __ldg(vsr4 + vb) : z4;
-    ++vb;
-    int s1 = vb < vb_end ? L.vsr_pos[vb] : 0x7FFFFFFF;
-    uint4 b1 = vb < vb_end ? __ldg(vsr4 + vb) : z4;
-    ++vb;
-    const uint32_t rsw = (uint32_t)(r & 7);
-    const uint4* cb1v = reinterpret_cast<const uint4*>(L.cb1);
-    auto load_f = [&](int kb, uint32_t* f) {
-      if (row_ok && kb < num_kb) load_fields<W, SPT>(codes_row, kb, jg, L.w, L.n_sub, f);
-      else for (int u = 0; u < SPT; ++u) f[u] = 0u;
-    };
-    auto load_cs = [&](int kb, uint4* c) {
-#pragma unroll
-      for (int u = 0; u < SPT; ++u)
-        c[u] = (has_cs && row_ok && kb < num_kb && kb * 8 + SPT * jg + u < L.n_sub)
-                   ? __ldg(reinterpret_cast<const uint4*>(L.cs + kb * 64 + cbeg + u * 8)) : z4;
-    };
-    auto gather = [&](int kb, const uint32_t* fl, uint4* g) {
-#pragma unroll
-      for (int u = 0; u < SPT; ++u) {
-        const int sv = kb * 8 + SPT * jg + u;
-        if (row_ok && kb < num_kb && sv < L.n_sub)
-          g[u] = ldg_nc_na(cb1v + (uint32_t)group_of(L, sv) * (uint32_t)L.k1 + (fl[u] & m1));
+    auto gather = [&](int kb, uint32_t f, uint32_t* g) {
+      const int sv = min(min(kb, last_kb) * 8 + svl, L.n_sub - 1);
+      const uint32_t* p = cb1w + ((size_t)((uint32_t)group_of(L, sv) * (uint32_t)L.k1 + (f & m1)) * 4 + hp * NW);
+      if constexpr (NW == 4) {
+        asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(g[0]), "=r"(g[1]), "=r"(g[2]), "=r"(g[3]) : "l"(p));
+      } else {
+        asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(g[0]), "=r"(g[1]) : "l"(p));
       }
     };
     bool ok = true;
     // One pipeline step for K-block kb: the loads for later K-blocks; the conversion of kb into
-    // registers, with the VSR blocks of the lane's sub-vectors put in their places; then, once
-    // every CTA's MMA is done with kb's slot, the stores, the CSR values over them and the
-    // arrival for the copier.  The callers rotate fixed register arrays through the roles, so no value in
+    // registers; then, once every CTA's MMA is done with kb's slot, the store and the arrival for
+    // the sparse warp.  The callers rotate fixed register arrays through the roles, so no value in
     // flight is ever copied.
-    auto step = [&](int kb, const uint4* g_cur, uint4* g_next, const uint32_t* f_next, uint32_t* f_load,
-                    const uint4* c_cur, uint4* c_load) {
-      load_f(kb + 6, f_load);
+    auto step = [&](int kb, const uint32_t* g_cur, uint32_t* g_next, uint32_t f_next, uint32_t& f_load,
+                    const uint32_t* c_cur, uint32_t* c_load) {
+      f_load = load_f(kb + 6);
       load_cs(kb + 3, c_load);
       gather(kb + 3, f_next, g_next);
-      uint32_t w4[SPT][4];
+      uint32_t w[NW];
+      const bool valid = row_ok && kb * 8 + svl < L.n_sub;
 #pragma unroll
-      for (int u = 0; u < SPT; ++u) {
-        const int sv = kb * 8 + SPT * jg + u;
-        w4[u][0] = w4[u][1] = w4[u][2] = w4[u][3] = 0u;
-        if (row_ok && sv < L.n_sub) {
-          const uint32_t cw[4] = {g_cur[u].x, g_cur[u].y, g_cur[u].z, g_cur[u].w};
-          const __half* ch = reinterpret_cast<const __half*>(&c_cur[u]);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const __half2 h2 = *reinterpret_cast<const __half2*>(&cw[q]);
-            float a0 = __low2float(h2) * rsc, a1 = __high2float(h2) * rsc;   // exact
-            if (has_cs) {
-              a0 = rto_mul_f32(a0, __half2float(ch[2 * q]));
-              a1 = rto_mul_f32(a1, __half2float(ch[2 * q + 1]));
-            }
-            w4[u][q] = (uint32_t)__half_as_ushort(__float2half_rn(a0)) |
-                       ((uint32_t)__half_as_ushort(__float2half_rn(a1)) << 16);
-          }
+      for (int q = 0; q < NW; ++q) {
+        const __half2 h2 = *reinterpret_cast<const __half2*>(&g_cur[q]);
+        float a0 = __low2float(h2) * rsc, a1 = __high2float(h2) * rsc;   // exact
+        if (has_cs) {
+          const __half2 c2 = *reinterpret_cast<const __half2*>(&c_cur[q]);
+          a0 = rto_mul_f32(a0, __low2float(c2));
+          a1 = rto_mul_f32(a1, __high2float(c2));
         }
-      }
-      const int col0 = kb * 64 + cbeg;                    // first column of this lane's sub-vectors
-      // VSR blocks of this row among the lane's sub-vectors replace them whole
-      while (s0 < kb * 8 + SPT * jg + SPT) {
-        const int u0 = s0 - (kb * 8 + SPT * jg);
-#pragma unroll
-        for (int u = 0; u < SPT; ++u)
-          if (u == u0) { w4[u][0] = b0.x; w4[u][1] = b0.y; w4[u][2] = b0.z; w4[u][3] = b0.w; }
-        s0 = s1; b0 = b1;
-        s1 = vb < vb_end ? L.vsr_pos[vb] : 0x7FFFFFFF;
-        b1 = vb < vb_end ? __ldg(vsr4 + vb) : z4;
-        ++vb;
+        const __half2 o = __floats2half2_rn(a0, a1);
+        w[q] = valid ? *reinterpret_cast<const uint32_t*>(&o) : 0u;
       }
       // the slot is free once every CTA's MMA is done with its previous K-block
       const int sa = kb % FA_STAGES;
       const bool mine = !*abort_flag && mbar_wait(smem_u32(&a_free[sa]), ((uint32_t)(kb / FA_STAGES) & 1u) ^ 1u, 3);
       if (!__all_sync(0xffffffffu, mine)) { *abort_flag = 1; ok = false; return; }
-      const uint32_t slot0 = smem_u32(ring_a + (size_t)sa * FA_BYTES);
-      const uint32_t slot = slot0 + (uint32_t)r * 128u;
-#pragma unroll
-      for (int u = 0; u < SPT; ++u) {
-        const uint32_t adr = slot + (((uint32_t)(SPT * jg + u) ^ rsw) << 4);
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(adr), "r"(w4[u][0]), "r"(w4[u][1]),
-                     "r"(w4[u][2]), "r"(w4[u][3])
+      const uint32_t adr = smem_u32(ring_a + (size_t)sa * FA_BYTES) + (uint32_t)r * 128u +
+                           ((((uint32_t)svl ^ rsw) << 4) | (uint32_t)(hp * 8));
+      if constexpr (NW == 4)
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(adr), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+                     "r"(w[3])
                      : "memory");
-      }
-      // sparse positions of this row inside the lane's columns take the stored value
-      for (int j = csr_col(); j < col0 + SPT * 8; j = csr_col()) {
-        if (j >= col0) {
-          const int k = j - kb * 64;                      // column inside the K-block
-          const uint32_t adr = slot + ((((uint32_t)k >> 3) ^ rsw) << 4) + (((uint32_t)k & 7u) << 1);
-          asm volatile("st.shared.u16 [%0], %1;" ::"r"(adr), "h"(csr_val()) : "memory");
-        }
-        csr_next();
-      }
+      else
+        asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(adr), "r"(w[0]), "r"(w[1]) : "memory");
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
       if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&own_full[sa])) : "memory");
     };
     // Array X_i holds the values of K-blocks congruent to i mod 4.
-    uint4 G0[SPT], G1[SPT], G2[SPT], G3[SPT];          // centroids in flight
-    uint32_t F0[SPT], F1[SPT], F2[SPT], F3[SPT];       // index fields
-    uint4 C0[SPT], C1[SPT], C2[SPT], C3[SPT];          // column scales
-    load_f(0, F0); load_f(1, F1); load_f(2, F2); load_f(3, F3);
+    uint32_t G0[NW], G1[NW], G2[NW], G3[NW];          // centroid parts in flight
+    uint32_t F0, F1, F2, F3;                           // index fields
+    uint32_t C0[NW], C1[NW], C2[NW], C3[NW];          // column scales
+    F0 = load_f(0); F1 = load_f(1); F2 = load_f(2); F3 = load_f(3);
     gather(0, F0, G0); gather(1, F1, G1); gather(2, F2, G2);
-    load_f(4, F0); load_f(5, F1);
+    F0 = load_f(4); F1 = load_f(5);
     load_cs(0, C0); load_cs(1, C1); load_cs(2, C2);
     for (int kb = 0; kb < num_kb && ok; kb += 4) {
       step(kb, G0, G3, F3, F2, C0, C3);
@@ -664,8 +658,9 @@ __global__ void __launch_bounds__(F_THREADS, 1)
       if (!ok || kb + 3 >= num_kb) break;
       step(kb + 3, G3, G2, F2, F1, C3, C2);
     }
-    // ---------------- epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31, accumulator (w - 3) / 4
-    const int q = warp & 3, half = (warp - 3) >> 2;
+    // ---------------- epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31; the four warps of
+    // group (w - PW0) / 4 read 128 columns of accumulator ((w - PW0) / 4) / 2
+    const int q = warp & 3, part = (warp - PW0) >> 2, half = part >> 1, c0 = (part & 1) * 128;
     const bool done = mbar_wait(smem_u32(acc_bar), 0, 4);
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     // tcgen05.ld is warp-wide: the whole warp reads, or none of it
@@ -673,7 +668,7 @@ __global__ void __launch_bounds__(F_THREADS, 1)
       const int64_t i = (int64_t)n0 + q * 32 + lane;
       const bool i_ok = i < L.n_out;
 #pragma unroll 1
-      for (int c = 0; c < 256; c += 32) {
+      for (int c = c0; c < c0 + 128; c += 32) {
         uint32_t v[32];
         tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(half * 256 + c), v);
         const int64_t mb = m0 + half * 256 + c;
@@ -780,7 +775,7 @@ static cudaError_t launch_vq_cs(const Layer& L, const CUtensorMap& mx, int64_t M
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3((unsigned)((groups + CS - 1) / CS * CS), (unsigned)((L.n_out + tc::F_ROWS - 1) / tc::F_ROWS));
-  cfg.blockDim = dim3(tc::F_THREADS);
+  cfg.blockDim = dim3(tc::f_threads(CS));
   cfg.dynamicSmemBytes = tc::F_SMEM_BYTES;
   cfg.stream = s;
   cfg.attrs = attr;

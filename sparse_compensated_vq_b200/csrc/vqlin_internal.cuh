@@ -39,6 +39,11 @@ struct Layer {
   const uint16_t* val;                  // [nnz] fp16 bits (exact replacement values)
   const float* delta;                   // [nnz] v - body, for the fused products
   const uint16_t* col16;                // [nnz] column ids as u16 when n_in <= 65536, else null
+  // The CSR entries by 64-column K-block, for the fused prefill GEMM (null unless it applies):
+  // entries of row i in K-block kb are kb_start[i*(n_kb+1)+kb] .. kb_start[i*(n_kb+1)+kb+1]-1, and
+  // kb_entry[e] = (col_e mod 64) << 16 | val_e.
+  const int32_t* kb_start;              // [n_out][n_kb + 1]
+  const uint32_t* kb_entry;             // [nnz]
   // VSR blocks (whole main-column sub-vectors, REPLACE): block b of row i is sub-vector
   // vsr_pos[b], b in [vsr_rp[i], vsr_rp[i+1]); vsr_val its fp16 values [nb][d]; vsr_delta the
   // fused-product form v - decoded body [nb][d] (fp32, 0 past the last main column)
