@@ -663,20 +663,62 @@ __global__ void __launch_bounds__(f_threads(CS), 1)
     const int q = warp & 3, part = (warp - PW0) >> 2, half = part >> 1, c0 = (part & 1) * 128;
     const bool done = mbar_wait(smem_u32(acc_bar), 0, 4);
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    // tcgen05.ld is warp-wide: the whole warp reads, or none of it
-    if (__all_sync(0xffffffffu, done && !*abort_flag) && half < halves) {
-      const int64_t i = (int64_t)n0 + q * 32 + lane;
-      const bool i_ok = i < L.n_out;
+    // the decision is the same for all 16 producer warps (tcgen05.ld is warp-wide, and the
+    // 16-bit path below has a barrier among them)
+    uint32_t go;
+    asm volatile(
+        "{\n .reg .pred p, r;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred r, 1, %2, p;\n selp.u32 %0, 1, 0, r;\n}"
+        : "=r"(go) : "r"((uint32_t)(done && !*abort_flag)), "n"(F_PROD_WARPS * 32) : "memory");
+    if (go && yt == VQLIN_F32) {
+      if (half < halves) {
+        const int64_t i = (int64_t)n0 + q * 32 + lane;
+        const bool i_ok = i < L.n_out;
 #pragma unroll 1
-      for (int c = c0; c < c0 + 128; c += 32) {
-        uint32_t v[32];
-        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(half * 256 + c), v);
-        const int64_t mb = m0 + half * 256 + c;
-        if (!i_ok) continue;
+        for (int c = c0; c < c0 + 128; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(half * 256 + c), v);
+          const int64_t mb = m0 + half * 256 + c;
+          if (!i_ok) continue;
 #pragma unroll
-        for (int jx = 0; jx < 32; ++jx) {
-          const int64_t m = mb + jx;
-          if (m < M) store_from_float(Y, yt, m * L.n_out + i, __uint_as_float(v[jx]));
+          for (int jx = 0; jx < 32; ++jx) {
+            const int64_t m = mb + jx;
+            if (m < M) reinterpret_cast<float*>(Y)[m * L.n_out + i] = __uint_as_float(v[jx]);
+          }
+        }
+      }
+    } else if (go) {
+      // 16-bit outputs: stage the CTA's 512 x 128 tile of Y in the activation ring (every MMA has
+      // completed, so it is free), Y-major, then write whole 256-byte row segments of Y
+      unsigned short* stage = reinterpret_cast<unsigned short*>(ring_b);   // [512][128]
+      const bool f16 = yt == VQLIN_F16;
+      if (half < halves) {
+#pragma unroll 1
+        for (int c = c0; c < c0 + 128; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(half * 256 + c), v);
+          unsigned short* sp = stage + (size_t)(half * 256 + c) * 128 + q * 32 + lane;
+#pragma unroll
+          for (int jx = 0; jx < 32; ++jx) {
+            const float f = __uint_as_float(v[jx]);
+            sp[jx * 128] = f16 ? __half_as_ushort(__float2half_rn(f)) : __bfloat16_as_ushort(__float2bfloat16_rn(f));
+          }
+        }
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(F_PROD_WARPS * 32) : "memory");
+      const int p = pw * 32 + lane, ch = p & 15;       // 16 threads per row of the tile, 8 columns each
+      const int64_t i0 = (int64_t)n0 + ch * 8;
+      const bool vec = i0 + 8 <= L.n_out && (L.n_out & 7) == 0 && (reinterpret_cast<uintptr_t>(Y) & 15) == 0;
+#pragma unroll 4
+      for (int ml = p >> 4; ml < 512; ml += 32) {
+        const int64_t m = m0 + ml;
+        if (m >= M) break;
+        const unsigned short* sp = stage + (size_t)ml * 128 + ch * 8;
+        unsigned short* yp = reinterpret_cast<unsigned short*>(Y) + m * L.n_out + i0;
+        if (vec) {
+          *reinterpret_cast<uint4*>(yp) = *reinterpret_cast<const uint4*>(sp);
+        } else {
+          for (int t = 0; t < 8; ++t)
+            if (i0 + t < L.n_out) yp[t] = sp[t];
         }
       }
     }
