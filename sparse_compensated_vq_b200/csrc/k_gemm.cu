@@ -689,6 +689,7 @@ __global__ void __launch_bounds__(f_threads(CS), 1)
     } else if (go) {
       // 16-bit outputs: stage the CTA's 512 x 128 tile of Y in the activation ring (every MMA has
       // completed, so it is free), Y-major, then write whole 256-byte row segments of Y
+      static_assert((size_t)FB_STAGES * FB_BYTES >= 512 * 128 * 2, "the output tile fits the activation ring");
       unsigned short* stage = reinterpret_cast<unsigned short*>(ring_b);   // [512][128]
       const bool f16 = yt == VQLIN_F16;
       if (half < halves) {
