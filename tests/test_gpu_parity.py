@@ -328,6 +328,43 @@ def test_gemm_fused_cluster_formats(vq, t, M):
     G.assert_close(G.to_f64(Y), oracle.gemv_f64(L, synth.bits_to_f64(Xb, "f16")), "f32", "fused gemm t=%d M=%d" % (t, M))
 
 
+@pytest.mark.parametrize("M", [300, 1100])
+@pytest.mark.parametrize("ydt", ["f16", "bf16"])
+def test_gemm_fused_16bit_outputs(vq, M, ydt):
+    """16-bit outputs of the fused prefill are staged through shared memory and written as row
+    segments of Y; n_out = 300 (not a multiple of 8) takes the element-wise tail of that write,
+    M = 1100 leaves CTAs past the last activation row."""
+    import torch
+    rng = np.random.default_rng(4500 + M)
+    L = synth.random_layer(rng, 300, 200, 8, 256, 8, col_scale=True, cb_std=0.3, nnz=700, outlier_scale=1.0)
+    Xb = synth.activations(rng, M, L.n_in, "f16")
+    m = vq.VQLinear(L)
+    Y = m.gemm(G.torch_x(Xb, "f16"), out_dtype=G.torch_dtype(ydt))
+    torch.cuda.synchronize()
+    assert vq.device_error() == 0
+    G.assert_close(G.to_f64(Y), oracle.gemv_f64(L, synth.bits_to_f64(Xb, "f16")), ydt, "fused gemm %s M=%d" % (ydt, M))
+
+
+@pytest.mark.parametrize("M", [600, 2100])
+def test_gemm_fused_dense_sparse_part(vq, M):
+    """Rows with many CSR entries in one 64-column block (more than the sparse warp's four
+    prefetched ones) and many VSR blocks, through the fused prefill: 25% of the elements are CSR
+    entries and a third of the remaining sub-vectors VSR blocks."""
+    import torch
+    rng = np.random.default_rng(4600 + M)
+    n_out, n_in = 140, 264
+    L = synth.random_layer(rng, n_out, n_in, 8, 256, 8, col_scale=True, cb_std=0.3,
+                           nnz=n_out * n_in // 4, outlier_scale=1.0, vsr_blocks=n_out * (n_in // 8) // 8)
+    Xb = synth.activations(rng, M, L.n_in, "f16")
+    m = vq.VQLinear(L)
+    n0 = vq.vqlin_kernel_launches()
+    Y = m.gemm(G.torch_x(Xb, "f16"), out_dtype=torch.float32)
+    assert vq.vqlin_kernel_launches() - n0 == 1
+    torch.cuda.synchronize()
+    assert vq.device_error() == 0
+    G.assert_close(G.to_f64(Y), oracle.gemv_f64(L, synth.bits_to_f64(Xb, "f16")), "f32", "fused gemm dense sparse M=%d" % M)
+
+
 def test_gemm_prefill_sampled_rows(vq):
     L, Xb = G.workload("prefill")
     Y = run_gemm(vq, L, Xb, "bf16", "bf16")
