@@ -274,8 +274,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 // Sharing the weight tile.  The CS CTAs of a thread-block cluster (CS = 2 up to 1024 activation
 // rows, 4 beyond) own the same 128 weight rows and different 512-row activation groups (a CTA past
 // the last activation row still converts and shares its part).  Each converts only its 128 / CS
-// rows of every weight K-block into its own slot, and one thread copies them into the same slot
-// of each peer (cp.async.bulk shared::cta -> shared::cluster, completing on the peer's slot
+// rows of every weight K-block into its own slot, and its sparse warps copy them into the same
+// slot of each peer (cp.async.bulk shared::cta -> shared::cluster, completing on the peer's slot
 // barrier).  So every weight element is gathered and converted once per 512 * CS activation rows.
 // A slot is rewritten only when every CTA's MMA has finished with it: the MMA returns a slot with
 // one tcgen05.commit multicast to the slot's "cluster free" barrier in every CTA of the cluster.
@@ -303,8 +303,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 //               TMA 128B-swizzle load makes) and makes the writes visible to the async proxy
 //               (fence.proxy.async).  The weight tile is therefore bit for bit the dequantised W.
 // Every mbarrier wait is bounded (1 s); on expiry the kernel records an error code, stops,
-// waits (bounded) for its own copies, frees TMEM and returns.  Every thread reaches the cluster
-// barriers at start and end.
+// waits (bounded) for its own TMA loads, frees TMEM and returns.  Every thread reaches the
+// cluster barriers at start and end.
 constexpr int FA_STAGES = 4, FB_STAGES = 5;
 constexpr int FA_BYTES = 128 * 64 * 2;             // 16 KB weight slot
 constexpr int FB_BYTES = 256 * 64 * 2;             // 32 KB activation half-slot
@@ -313,14 +313,6 @@ constexpr int F_PROD_WARPS = 16;
 __host__ __device__ constexpr int f_threads(int cs) { return (2 + 4 / cs + F_PROD_WARPS) * 32; }
 constexpr int F_ROWS = 128, F_XROWS = 512;
 constexpr size_t F_SMEM_BYTES = 1024 + (size_t)FA_STAGES * FA_BYTES + (size_t)FB_STAGES * FB_BYTES + 256;
-
-// 16-byte global load that is not kept in L1 (a centroid gather: no reuse worth caching)
-__device__ __forceinline__ uint4 ldg_nc_na(const uint4* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-  return v;
-}
 
 // fp32 product rounded to odd: toward zero, last bit forced to 1 when inexact (the exact error
 // comes from a fused multiply-add).  Rounding that to fp16 gives the correctly rounded product.
