@@ -365,6 +365,22 @@ def test_gemm_fused_dense_sparse_part(vq, M):
     G.assert_close(G.to_f64(Y), oracle.gemv_f64(L, synth.bits_to_f64(Xb, "f16")), "f32", "fused gemm dense sparse M=%d" % M)
 
 
+def test_gemm_fused_more_ctas_than_sms(vq):
+    """A fused prefill whose grid (11 weight tiles x 16 activation groups = 176 CTAs in clusters
+    of 4) does not fit on the GPU at once, so clusters run in more than one wave."""
+    import torch
+    rng = np.random.default_rng(4700)
+    L = synth.random_layer(rng, 1300, 136, 8, 256, 8, col_scale=True, cb_std=0.3, nnz=900, outlier_scale=1.0)
+    M = 8192
+    Xb = synth.activations(rng, M, L.n_in, "f16")
+    m = vq.VQLinear(L)
+    Y = m.gemm(G.torch_x(Xb, "f16"), out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert vq.device_error() == 0
+    rows = np.sort(rng.choice(M, 256, replace=False))
+    G.assert_close(G.to_f64(Y)[rows], oracle.gemv_f64(L, synth.bits_to_f64(Xb[rows], "f16")), "f32", "fused gemm 176 CTAs")
+
+
 def test_gemm_prefill_sampled_rows(vq):
     L, Xb = G.workload("prefill")
     Y = run_gemm(vq, L, Xb, "bf16", "bf16")
